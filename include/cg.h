@@ -1,0 +1,208 @@
+/*
+ * cg.h -- C ABI of libcg, a B200 (sm_100a) implementation of the Codec-Gauge
+ * cache-coordinate codec round trip on KV tensors.
+ *
+ * Source method: "Codec-Gauge: Learning Compression-Friendly Gauges for
+ * Transformer KV Caches" (arXiv 2607.20538).  A small orthogonal gauge
+ * G = exp(A - A^T) per (layer, K/V, head, channel group) maps cached keys and
+ * values into coordinates a fixed low-bit backend preserves better; it is
+ * applied before quantization and inverted (G^T) before attention.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every pointer argument named *_dev is DEVICE memory owned by the
+ *           caller; the library never allocates, frees or retains device
+ *           memory between calls (a caller-sized workspace is passed where a
+ *           kernel needs scratch).  Descriptors are HOST structs read during
+ *           the call only.
+ * Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *           work is enqueued asynchronously; nothing synchronizes the host.
+ * Layout.   The KV cache is bf16 [L][2][B][H][T][d], row-major, s = 0 keys and
+ *           s = 1 values, T the token capacity.  Gauges are fp32
+ *           [L][2][H][R][g][g] with R = d / g, row-major, y_i = sum_j G[i][j] x_j
+ *           for the g-vector x of one token in one channel group (shared over
+ *           the batch).
+ * Errors.   Argument errors (null or misaligned pointers, unsupported sizes,
+ *           token ranges off the block grid) return CG_ERR_INVALID or
+ *           CG_ERR_UNSUPPORTED before anything is enqueued, and leave every
+ *           output untouched.  A failed launch returns CG_ERR_CUDA.  Kernels
+ *           that wait on asynchronous copies bound every wait; a wait that runs
+ *           out records a device status word that cg_sync_status() reports as
+ *           CG_ERR_TIMEOUT.  Inputs must be finite: NaN or Inf values give
+ *           unspecified codes (no fault).
+ * Alignment. All device pointers must be 16-byte aligned.
+ * Threads.  Calls are re-entrant; concurrent calls on different streams are
+ *           independent (apart from the shared status word).
+ */
+#ifndef CG_H_
+#define CG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CG_OK = 0,
+  CG_ERR_INVALID = 1,     /* bad argument: null, misaligned, out of range   */
+  CG_ERR_UNSUPPORTED = 2, /* valid request this build has no kernel for     */
+  CG_ERR_CUDA = 3,        /* launch or runtime error                        */
+  CG_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out             */
+} cg_status;
+
+typedef enum {
+  CG_QUANT_BLOCK_UNIFORM = 0, /* one min/max range per T_b x W block          */
+  CG_QUANT_KIVI = 1           /* keys per channel, values per token           */
+} cg_quant_mode;
+
+/* Shape of a KV cache: K_l, V_l in R^{B x H x T x d} for l = 1..L
+ * (Codec-Gauge, Problem statement and overview).  `tokens` is the capacity T
+ * of the buffer; encode/decode take a token range inside it. */
+typedef struct {
+  int32_t layers;  /* L */
+  int32_t batch;   /* B */
+  int32_t heads;   /* H (KV heads) */
+  int32_t tokens;  /* T (capacity), a multiple of 32 */
+  int32_t d_head;  /* d: 64 or 128 */
+} cg_kv_desc;
+
+/* Codec settings.
+ *   g           gauge group size: 8, 16, 32 (grouped) or d_head (full head)
+ *               (Codec-Gauge, Method: g = 8, 16, 32 and full-head gauges).
+ *   bits        bits per value: 2, 3, 4, 6 or 8 (Experimental setup).
+ *   tb          token block T_b of the block-uniform ranges: 16.
+ *   range_cols  W, channels per block-uniform range: g (default) or d_head
+ *               (the page's "one range per T_b x d_l block").
+ *   mode        cg_quant_mode.
+ *   kivi_key_tokens, kivi_val_channels: KIVI group sizes, both 32.
+ */
+typedef struct {
+  int32_t g;
+  int32_t bits;
+  int32_t tb;
+  int32_t range_cols;
+  int32_t mode;
+  int32_t kivi_key_tokens;
+  int32_t kivi_val_channels;
+} cg_codec_desc;
+
+/* Buffer sizes of an encoded cache (whole capacity T).  The zero-point and
+ * scale arrays are fp16 with scale_count entries each, so the actual
+ * bits/value is 8 (code_bytes + 4 scale_count) / N_KV with
+ * N_KV = sum_l 2 B H T d (Codec-Gauge, Problem statement; Experimental setup:
+ * actual bits/value computed from measured bytes). */
+typedef struct {
+  uint64_t code_bytes;
+  uint64_t scale_count;
+} cg_sizes;
+
+/* Spectral-statistics settings (Codec-Gauge, Method: T_b = 16,
+ * lambda_f = 1.0, lambda_r = 0.02, tau = 0.04 for every checkpoint). */
+typedef struct {
+  int32_t tb;        /* token block of the DCT: 16 */
+  int32_t g;         /* group size of G when a gauge is fused, else 0 */
+  int32_t x_is_fp32; /* 1: x is fp32, 0: x is bf16 */
+  float lambda_f;
+  float lambda_r;
+  float tau;
+} cg_stats_desc;
+
+/* Host only.  Fills *out with the exact byte / entry counts of the encoded
+ * buffers for `kv` and `codec`; validates both descriptors.
+ *   block-uniform: code_bytes = L 2 B H T d bits / 8,
+ *                  scale_count = L 2 B H (T / tb) (d / W)
+ *   KIVI:          code_bytes as above, scale_count = L 2 B H T d / 32 */
+cg_status cg_sizes_for(const cg_kv_desc* kv, const cg_codec_desc* codec, cg_sizes* out);
+
+/* G = exp(A - A^T) for n_mats independent g x g matrices
+ * (Codec-Gauge, Method: gauge parameterization; the displayed equation is
+ * missing from the page, which names exp(.) and the skew matrix A - A^T).
+ *   A_dev, G_dev : fp32 [n_mats][g][g], row-major, may not alias.
+ *   g            : 2 .. 128.
+ * fp32 scaling and squaring with a Taylor core; G is orthogonal to about 1e-6.
+ * One thread block per matrix. */
+cg_status cg_gauge_build(const float* A_dev, float* G_dev, int32_t n_mats, int32_t g, void* stream);
+
+/* Fused gauge + quantize + pack for tokens [t0, t0 + nt) of every
+ * (layer, K/V, batch, head)
+ * (Codec-Gauge, Figure 1 / Backend compatibility: the gauge is applied at the
+ * KV tensor interface before quantization; Experimental setup: block-uniform
+ * and KIVI-style backends).
+ *   kv_dev      bf16 [L][2][B][H][T][d]                         (input)
+ *   G_dev       fp32 [L][2][H][d/g][g][g]                        (input)
+ *   codes_dev   uint8, cg_sizes.code_bytes for the whole capacity (output)
+ *   scales_dev, zeros_dev  fp16, cg_sizes.scale_count each       (output)
+ *   gauged_dev  optional fp32 [L][2][B][H][T][d]: the gauged values the
+ *               quantizer saw (NULL to skip; costs 4 B/value of traffic)
+ * Only the blocks covering [t0, t0 + nt) are written.  t0 and nt must be
+ * multiples of tb (block-uniform) or of 32 (KIVI).
+ * Block-uniform layout: codes [L][2][B][H][T/tb][d/W][tb*W*bits/8], element
+ * i = t_local*W + c_local of a block holding bits [i*bits, i*bits + bits) of a
+ * little-endian bit stream; scales / zeros [L][2][B][H][T/tb][d/W].
+ * KIVI layout: keys (s = 0) codes [..][T/32][d][32*bits/8] (token-ascending),
+ * values (s = 1) codes [..][T][d/32][32*bits/8] (channel-ascending); scales /
+ * zeros [..][T/32][d] and [..][T][d/32].
+ * Per range: z = fp16(min), s = fp16(fl32(fl32(max - min) / (2^b - 1))),
+ * q = clamp(rne(fl32(fl32(y - z) * fl32(1/s))), 0, 2^b - 1), q = 0 if s = 0.
+ * Gauged values: for g < d each y_i is the fp32 fused-multiply-add chain over
+ * j = 0..g-1 in index order (bit-reproducible); for g = d the contraction runs
+ * on the tensor cores with G rounded to bf16 and fp32 accumulation. */
+cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec,
+                    const void* kv_dev, const float* G_dev, int32_t t0, int32_t nt,
+                    uint8_t* codes_dev, void* scales_dev, void* zeros_dev,
+                    float* gauged_dev, void* stream);
+
+/* Fused unpack + dequantize + inverse gauge for tokens [t0, t0 + nt)
+ * (Codec-Gauge, Figure 1: the inverse gauge restores the KV state before
+ * attention; Method: explicit key/value recovery, charged in timing).
+ *   x_hat = G^T (s q + z) per token and group, written as bf16 (RNE) into
+ *   kv_out_dev [L][2][B][H][T][d] (other tokens untouched).
+ * Buffers and layouts as in cg_encode.  G for g = d is rounded to bf16. */
+cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec,
+                    const uint8_t* codes_dev, const void* scales_dev, const void* zeros_dev,
+                    const float* G_dev, int32_t t0, int32_t nt, void* kv_out_dev, void* stream);
+
+/* Workspace bytes cg_spectral_stats needs for this shape (host only). */
+cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* st,
+                                     int32_t want_grad, uint64_t* bytes);
+
+/* Gauge-training statistics (Codec-Gauge, Method: frequency-distribution
+ * objective).  Every T_b x d token-channel block of X' = G X (or of x itself
+ * when G_dev is NULL) gets a 2-D orthonormal DCT-II U = C_Tb X' C_d^T; per
+ * block
+ *   L_freq = sum r_uv U_uv^2 / sum U_uv^2  (0 for an all-zero block),
+ *   r_uv = sqrt((u/(T_b-1))^2 + (v/(d-1))^2) / sqrt(2),
+ *   L_rate = mean log(1 + |U_uv| / tau)    (assumed form: the page's equation
+ *                                           is truncated),
+ * and L = lambda_f mean(L_freq) + lambda_r mean(L_rate).
+ *   x_dev        bf16 or fp32 [L][2][B][H][T][d]
+ *   G_dev        fp32 [L][2][H][d/g][g][g] or NULL (x already gauged)
+ *   lfreq_dev, lrate_dev  fp32 [L][2][B][H][T/tb]              (output)
+ *   totals_dev   fp64 [4]: sum L_freq, sum L_rate, n_blocks, L  (output)
+ *   dG_dev       fp32 [L][2][H][d/g][g][g] = dL/dG, or NULL; requires G_dev
+ *   workspace_dev / workspace_bytes: at least cg_spectral_workspace_size().
+ * Reductions run in a fixed order: results are deterministic for a given
+ * shape. */
+cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st,
+                            const void* x_dev, const float* G_dev,
+                            float* lfreq_dev, float* lrate_dev, double* totals_dev,
+                            float* dG_dev, void* workspace_dev, uint64_t workspace_bytes,
+                            void* stream);
+
+/* Synchronizes `stream`, then reports (and clears) the device status word:
+ * CG_ERR_TIMEOUT if a bounded wait ran out since the last check, CG_ERR_CUDA on
+ * a pending CUDA error, else CG_OK. */
+cg_status cg_sync_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* cg_status_string(cg_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t cg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CG_H_ */

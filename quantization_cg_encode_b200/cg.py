@@ -1,0 +1,195 @@
+"""Thin Python binding of libcg (C ABI in include/cg.h).
+
+Argument marshalling only: every function checks the torch tensors it is given
+(device, dtype, contiguity, size), passes their raw device pointers and the
+current CUDA stream to the C entry point of the same name, and raises on a
+non-OK status.  All computation happens in the CUDA library; there is no
+fallback of any kind.  torch is used for device memory and streams only.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcg.so")
+
+CG_OK, CG_ERR_INVALID, CG_ERR_UNSUPPORTED, CG_ERR_CUDA, CG_ERR_TIMEOUT = range(5)
+BLOCK_UNIFORM, KIVI = 0, 1
+
+# Every symbol include/cg.h declares.
+EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
+           "cg_spectral_stats", "cg_sync_status", "cg_status_string", "cg_version")
+
+
+class KvDesc(ctypes.Structure):
+    _fields_ = [("layers", ctypes.c_int32), ("batch", ctypes.c_int32), ("heads", ctypes.c_int32),
+                ("tokens", ctypes.c_int32), ("d_head", ctypes.c_int32)]
+
+
+class CodecDesc(ctypes.Structure):
+    _fields_ = [("g", ctypes.c_int32), ("bits", ctypes.c_int32), ("tb", ctypes.c_int32),
+                ("range_cols", ctypes.c_int32), ("mode", ctypes.c_int32),
+                ("kivi_key_tokens", ctypes.c_int32), ("kivi_val_channels", ctypes.c_int32)]
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [("code_bytes", ctypes.c_uint64), ("scale_count", ctypes.c_uint64)]
+
+
+class StatsDesc(ctypes.Structure):
+    _fields_ = [("tb", ctypes.c_int32), ("g", ctypes.c_int32), ("x_is_fp32", ctypes.c_int32),
+                ("lambda_f", ctypes.c_float), ("lambda_r", ctypes.c_float), ("tau", ctypes.c_float)]
+
+
+class CgError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libcg.  Raises if the library has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libcg.so not found at %s: build it with `python -m quantization_cg_encode_b200.build`"
+                              % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64
+        L.cg_sizes_for.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), ctypes.POINTER(Sizes)]
+        L.cg_gauge_build.argtypes = [vp, vp, i32, i32, vp]
+        L.cg_encode.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, i32, i32, vp, vp, vp, vp, vp]
+        L.cg_decode.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, vp, vp, i32, i32, vp, vp]
+        L.cg_spectral_workspace_size.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(StatsDesc), i32,
+                                                 ctypes.POINTER(u64)]
+        L.cg_spectral_stats.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(StatsDesc), vp, vp, vp, vp, vp, vp,
+                                        vp, u64, vp]
+        L.cg_sync_status.argtypes = [vp]
+        L.cg_status_string.argtypes = [ctypes.c_int]
+        L.cg_status_string.restype = ctypes.c_char_p
+        L.cg_version.restype = ctypes.c_int32
+        for name in ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
+                     "cg_spectral_stats", "cg_sync_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().cg_status_string(int(status)).decode()
+
+
+def _check(status, where):
+    if status != CG_OK:
+        raise CgError(status, where)
+
+
+def _ptr(t, dtype, name, numel=None):
+    """Device pointer of a contiguous CUDA tensor of the given dtype (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if numel is not None and t.numel() < numel:
+        raise ValueError("%s holds %d elements, needs %d" % (name, t.numel(), numel))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def kv_desc(layers, batch, heads, tokens, d_head):
+    return KvDesc(layers, batch, heads, tokens, d_head)
+
+
+def codec_desc(g=16, bits=4, tb=16, range_cols=None, mode=BLOCK_UNIFORM, kivi_key_tokens=32, kivi_val_channels=32):
+    return CodecDesc(g, bits, tb, g if range_cols is None else range_cols, mode, kivi_key_tokens, kivi_val_channels)
+
+
+def kv_desc_of(kv):
+    """KvDesc of a [L, 2, B, H, T, d] tensor."""
+    L, two, B, H, T, d = kv.shape
+    assert two == 2
+    return KvDesc(L, B, H, T, d)
+
+
+def cg_sizes_for(kvd, codec):
+    out = Sizes()
+    _check(lib().cg_sizes_for(ctypes.byref(kvd), ctypes.byref(codec), ctypes.byref(out)), "cg_sizes_for")
+    return int(out.code_bytes), int(out.scale_count)
+
+
+def gauge_numel(kvd, g):
+    """Elements of a [L, 2, H, d/g, g, g] gauge array."""
+    return kvd.layers * 2 * kvd.heads * kvd.d_head * g
+
+
+def alloc_encoded(kvd, codec, device="cuda"):
+    """Caller-owned output buffers (codes uint8, scales fp16, zeros fp16)."""
+    cb, sc = cg_sizes_for(kvd, codec)
+    return (torch.zeros(cb, dtype=torch.uint8, device=device),
+            torch.zeros(sc, dtype=torch.float16, device=device),
+            torch.zeros(sc, dtype=torch.float16, device=device))
+
+
+def cg_gauge_build(A, G, stream=None):
+    """G = exp(A - A^T) for A of shape [..., g, g] (fp32)."""
+    g = A.shape[-1]
+    n = A.numel() // (g * g)
+    _check(lib().cg_gauge_build(_ptr(A, torch.float32, "A"), _ptr(G, torch.float32, "G", A.numel()), n, g,
+                                _stream(stream)), "cg_gauge_build")
+    return G
+
+
+def cg_encode(kvd, codec, kv, G, t0, nt, codes, scales, zeros, gauged=None, stream=None):
+    n = kvd.layers * 2 * kvd.batch * kvd.heads * kvd.tokens * kvd.d_head
+    cb, sc = cg_sizes_for(kvd, codec)
+    _check(lib().cg_encode(ctypes.byref(kvd), ctypes.byref(codec), _ptr(kv, torch.bfloat16, "kv", n),
+                           _ptr(G, torch.float32, "G", gauge_numel(kvd, codec.g)),
+                           int(t0), int(nt), _ptr(codes, torch.uint8, "codes", cb),
+                           _ptr(scales, torch.float16, "scales", sc), _ptr(zeros, torch.float16, "zeros", sc),
+                           _ptr(gauged, torch.float32, "gauged", n), _stream(stream)), "cg_encode")
+
+
+def cg_decode(kvd, codec, codes, scales, zeros, G, t0, nt, kv_out, stream=None):
+    n = kvd.layers * 2 * kvd.batch * kvd.heads * kvd.tokens * kvd.d_head
+    cb, sc = cg_sizes_for(kvd, codec)
+    _check(lib().cg_decode(ctypes.byref(kvd), ctypes.byref(codec), _ptr(codes, torch.uint8, "codes", cb),
+                           _ptr(scales, torch.float16, "scales", sc), _ptr(zeros, torch.float16, "zeros", sc),
+                           _ptr(G, torch.float32, "G", gauge_numel(kvd, codec.g)), int(t0), int(nt), _ptr(kv_out, torch.bfloat16, "kv_out", n),
+                           _stream(stream)), "cg_decode")
+
+
+def cg_spectral_workspace_size(kvd, st, want_grad):
+    out = ctypes.c_uint64()
+    _check(lib().cg_spectral_workspace_size(ctypes.byref(kvd), ctypes.byref(st), int(bool(want_grad)),
+                                            ctypes.byref(out)), "cg_spectral_workspace_size")
+    return int(out.value)
+
+
+def cg_spectral_stats(kvd, st, x, G, lfreq, lrate, totals, dG=None, workspace=None, stream=None):
+    xdt = torch.float32 if st.x_is_fp32 else torch.bfloat16
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().cg_spectral_stats(ctypes.byref(kvd), ctypes.byref(st), _ptr(x, xdt, "x"), _ptr(G, torch.float32, "G"),
+                                   _ptr(lfreq, torch.float32, "lfreq"), _ptr(lrate, torch.float32, "lrate"),
+                                   _ptr(totals, torch.float64, "totals", 4), _ptr(dG, torch.float32, "dG"),
+                                   None if workspace is None else ctypes.c_void_p(workspace.data_ptr()),
+                                   ws_bytes, _stream(stream)), "cg_spectral_stats")
+
+
+def cg_sync_status(stream=None):
+    _check(lib().cg_sync_status(_stream(stream)), "cg_sync_status")
+
+
+def cg_version():
+    return int(lib().cg_version())

@@ -1,0 +1,213 @@
+// C ABI of libcg (declared in include/cg.h): argument validation, buffer
+// sizes, kernel dispatch and the device status word.
+#include <cstring>
+
+#include "cg_kernels.cuh"
+
+namespace cg {
+__device__ unsigned int g_status = 0;
+}
+
+using namespace cg;
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 6 || b == 8; }
+
+cg_status check_kv(const cg_kv_desc* kv) {
+  if (!kv) return CG_ERR_INVALID;
+  if (kv->layers <= 0 || kv->batch <= 0 || kv->heads <= 0 || kv->tokens <= 0 || kv->d_head <= 0) return CG_ERR_INVALID;
+  if (kv->tokens % 32 != 0) return CG_ERR_INVALID;
+  if (kv->d_head != 64 && kv->d_head != 128) return CG_ERR_UNSUPPORTED;
+  return CG_OK;
+}
+
+cg_status check_codec(const cg_kv_desc* kv, const cg_codec_desc* c) {
+  cg_status st = check_kv(kv);
+  if (st != CG_OK) return st;
+  if (!c) return CG_ERR_INVALID;
+  const int d = kv->d_head;
+  if (c->g <= 0 || d % c->g != 0) return CG_ERR_INVALID;
+  if (c->g != 8 && c->g != 16 && c->g != 32 && c->g != d) return CG_ERR_UNSUPPORTED;
+  if (!valid_bits(c->bits)) return CG_ERR_UNSUPPORTED;
+  if (c->mode == CG_QUANT_BLOCK_UNIFORM) {
+    if (c->tb != 16) return CG_ERR_UNSUPPORTED;
+    if (c->range_cols <= 0 || c->range_cols % c->g != 0 || d % c->range_cols != 0) return CG_ERR_INVALID;
+    if (c->range_cols != c->g && c->range_cols != d) return CG_ERR_UNSUPPORTED;
+  } else if (c->mode == CG_QUANT_KIVI) {
+    if (c->kivi_key_tokens != 32 || c->kivi_val_channels != 32) return CG_ERR_UNSUPPORTED;
+    if (c->g > 32) return CG_ERR_UNSUPPORTED;
+  } else {
+    return CG_ERR_INVALID;
+  }
+  return CG_OK;
+}
+
+cg_status check_range(const cg_kv_desc* kv, const cg_codec_desc* c, int t0, int nt) {
+  const int step = c->mode == CG_QUANT_KIVI ? 32 : c->tb;
+  if (t0 < 0 || nt < 0 || (long long)t0 + nt > kv->tokens) return CG_ERR_INVALID;
+  if (t0 % step != 0 || nt % step != 0) return CG_ERR_INVALID;
+  return CG_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+KvGeom geom(const cg_kv_desc* kv) { return KvGeom{kv->layers, kv->batch, kv->heads, kv->tokens, kv->d_head}; }
+
+cg_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CG_OK : CG_ERR_CUDA; }
+
+// Device address of the status word on the current device (looked up once
+// per device; a host-side symbol is not a device address).
+unsigned int* status_word() {
+  static unsigned int* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, cg::g_status) != cudaSuccess) return nullptr;
+    addr[dev] = (unsigned int*)p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+cg_status cg_sizes_for(const cg_kv_desc* kv, const cg_codec_desc* codec, cg_sizes* out) {
+  cg_status st = check_codec(kv, codec);
+  if (st != CG_OK) return st;
+  if (!out) return CG_ERR_INVALID;
+  const uint64_t heads = (uint64_t)kv->layers * 2 * kv->batch * kv->heads;
+  const uint64_t n = heads * kv->tokens * kv->d_head;
+  out->code_bytes = n * codec->bits / 8;
+  if (codec->mode == CG_QUANT_BLOCK_UNIFORM)
+    out->scale_count = heads * (kv->tokens / codec->tb) * (kv->d_head / codec->range_cols);
+  else
+    out->scale_count = n / 32;
+  return CG_OK;
+}
+
+cg_status cg_gauge_build(const float* A_dev, float* G_dev, int32_t n_mats, int32_t g, void* stream) {
+  if (n_mats < 0 || g < 2 || g > 128) return CG_ERR_INVALID;
+  if (n_mats == 0) return CG_OK;
+  if (!A_dev || !G_dev || !aligned16(A_dev) || !aligned16(G_dev) || A_dev == G_dev) return CG_ERR_INVALID;
+  return from_cuda(launch_gauge_build(A_dev, G_dev, n_mats, g, (cudaStream_t)stream));
+}
+
+cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec, const void* kv_dev, const float* G_dev, int32_t t0,
+                    int32_t nt, uint8_t* codes_dev, void* scales_dev, void* zeros_dev, float* gauged_dev, void* stream) {
+  cg_status st = check_codec(kv, codec);
+  if (st != CG_OK) return st;
+  st = check_range(kv, codec, t0, nt);
+  if (st != CG_OK) return st;
+  if (!kv_dev || !G_dev || !codes_dev || !scales_dev || !zeros_dev) return CG_ERR_INVALID;
+  if (!aligned16(kv_dev) || !aligned16(G_dev) || !aligned16(codes_dev) || !aligned16(scales_dev) ||
+      !aligned16(zeros_dev) || (gauged_dev && !aligned16(gauged_dev)))
+    return CG_ERR_INVALID;
+  if (nt == 0) return CG_OK;
+  CodecArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.k = geom(kv);
+  a.g = codec->g;
+  a.bits = codec->bits;
+  a.W = codec->range_cols;
+  a.kivi = codec->mode == CG_QUANT_KIVI;
+  a.t0 = t0;
+  a.nt = nt;
+  a.kv = (const uint16_t*)kv_dev;
+  a.G = G_dev;
+  a.codes = codes_dev;
+  a.scales = (uint16_t*)scales_dev;
+  a.zeros = (uint16_t*)zeros_dev;
+  a.gauged = gauged_dev;
+  a.status = status_word();
+  if (!a.status) return CG_ERR_CUDA;
+  if (a.kivi || a.g == kv->d_head) return CG_ERR_UNSUPPORTED;
+  return from_cuda(launch_group_codec(a, true, num_sms(), (cudaStream_t)stream));
+}
+
+cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec, const uint8_t* codes_dev, const void* scales_dev,
+                    const void* zeros_dev, const float* G_dev, int32_t t0, int32_t nt, void* kv_out_dev, void* stream) {
+  cg_status st = check_codec(kv, codec);
+  if (st != CG_OK) return st;
+  st = check_range(kv, codec, t0, nt);
+  if (st != CG_OK) return st;
+  if (!codes_dev || !scales_dev || !zeros_dev || !G_dev || !kv_out_dev) return CG_ERR_INVALID;
+  if (!aligned16(codes_dev) || !aligned16(scales_dev) || !aligned16(zeros_dev) || !aligned16(G_dev) ||
+      !aligned16(kv_out_dev))
+    return CG_ERR_INVALID;
+  if (nt == 0) return CG_OK;
+  CodecArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.k = geom(kv);
+  a.g = codec->g;
+  a.bits = codec->bits;
+  a.W = codec->range_cols;
+  a.kivi = codec->mode == CG_QUANT_KIVI;
+  a.t0 = t0;
+  a.nt = nt;
+  a.G = G_dev;
+  a.codes_in = codes_dev;
+  a.scales_in = (const uint16_t*)scales_dev;
+  a.zeros_in = (const uint16_t*)zeros_dev;
+  a.kv_out = (uint16_t*)kv_out_dev;
+  a.status = status_word();
+  if (!a.status) return CG_ERR_CUDA;
+  if (a.kivi || a.g == kv->d_head) return CG_ERR_UNSUPPORTED;
+  return from_cuda(launch_group_codec(a, false, num_sms(), (cudaStream_t)stream));
+}
+
+cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* st, int32_t want_grad, uint64_t* bytes) {
+  (void)want_grad;
+  cg_status s = check_kv(kv);
+  if (s != CG_OK) return s;
+  if (!st || !bytes) return CG_ERR_INVALID;
+  return CG_ERR_UNSUPPORTED;
+}
+
+cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st, const void* x_dev, const float* G_dev,
+                            float* lfreq_dev, float* lrate_dev, double* totals_dev, float* dG_dev, void* workspace_dev,
+                            uint64_t workspace_bytes, void* stream) {
+  (void)x_dev; (void)G_dev; (void)lfreq_dev; (void)lrate_dev; (void)totals_dev; (void)dG_dev;
+  (void)workspace_dev; (void)workspace_bytes; (void)stream;
+  cg_status s = check_kv(kv);
+  if (s != CG_OK) return s;
+  if (!st) return CG_ERR_INVALID;
+  return CG_ERR_UNSUPPORTED;
+}
+
+cg_status cg_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return CG_ERR_CUDA;
+  unsigned int flag = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&flag, cg::g_status, sizeof(flag));
+  if (e != cudaSuccess) return CG_ERR_CUDA;
+  if (flag) {
+    e = cudaMemcpyToSymbol(cg::g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return CG_ERR_CUDA;
+    return CG_ERR_TIMEOUT;
+  }
+  return CG_OK;
+}
+
+const char* cg_status_string(cg_status s) {
+  switch (s) {
+    case CG_OK: return "ok";
+    case CG_ERR_INVALID: return "invalid argument";
+    case CG_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CG_ERR_CUDA: return "CUDA error";
+    case CG_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t cg_version(void) { return 100; }
+
+}  // extern "C"
