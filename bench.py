@@ -1,0 +1,352 @@
+"""Benchmark of the Codec-Gauge KV codec round trip on one or more B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--bits 4] [--impl cg|reference]
+
+One step = fused gauge + quantize + pack encode (cg_encode) followed by fused
+unpack + dequantize + inverse-gauge decode (cg_decode) of a Llama-3-8B-shaped
+GQA cache: 32 layers x {K, V} x 8 KV heads x 4096 tokens x d_head 128, batch 1,
+bf16 (268,435,456 values, 0.537 GB), gauge groups g = 16, block-uniform ranges
+of 16 tokens x 16 channels.  Inputs are seeded synthetic caches (AR(1) keys with
+lognormal channel scales and outlier channels, AR(1) values); the gauge is
+built on the device from A ~ N(0, 0.1^2) by cg_gauge_build before timing.
+
+Metric: KV GB/s = bf16 KV bytes (2 N) carried through encode + decode per
+second, summed over GPUs (each GPU runs its own replica: the codec has no
+cross-GPU exchange, so scaling is weak).  Per-kernel rates and the HBM roofline
+fraction of the dominant kernel come with it.  The working set (0.54 GB in,
+0.13 GB codes, 0.54 GB out) is far larger than the 126 MB L2, so no flush is
+needed between steps.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L, B, H, T, D = 32, 1, 8, 4096, 128
+G_GROUP = 16
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_cg(args):
+    import torch
+    import torch.distributed as dist
+    from quantization_cg_encode_b200 import cg, synth
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+
+    kvd = cg.kv_desc(L, B, H, T, D)
+    codec = cg.codec_desc(g=G_GROUP, bits=args.bits)
+    n_values = L * 2 * B * H * T * D
+    kv_bytes = 2 * n_values
+
+    with torch.cuda.stream(stream):
+        kv = synth.kv_cache(L, B, H, T, D, seed=rank, device=dev, n_outliers=4)
+        A = synth.gauge_params(L, H, D // G_GROUP, G_GROUP, sigma=0.1, seed=rank).to(dev)
+        G = torch.empty_like(A)
+        cg.cg_gauge_build(A, G, stream=stream)
+        codes, scales, zeros = cg.alloc_encoded(kvd, codec, device=dev)
+        out = torch.empty_like(kv)
+    stream.synchronize()
+
+    def step():
+        cg.cg_encode(kvd, codec, kv, G, 0, T, codes, scales, zeros, None, stream=stream)
+        cg.cg_decode(kvd, codec, codes, scales, zeros, G, 0, T, out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    cg.cg_sync_status(stream)
+
+    # --- timed region: K steps, events on the launching stream --------------------------
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for e0, e1, e2 in ev:
+            e0.record(stream)
+            cg.cg_encode(kvd, codec, kv, G, 0, T, codes, scales, zeros, None, stream=stream)
+            e1.record(stream)
+            cg.cg_decode(kvd, codec, codes, scales, zeros, G, 0, T, out, stream=stream)
+            e2.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    cg.cg_sync_status(stream)
+    total_ms = t_start.elapsed_time(t_end)
+    enc_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    dec_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+
+    # --- end to end through the C ABI with host buffers -------------------------------------
+    kv_host = kv.cpu().pin_memory()
+    out_host = torch.empty(kv.shape, dtype=kv.dtype, pin_memory=True)
+    kv_dev2 = torch.empty_like(kv)
+
+    def e2e_step():
+        kv_dev2.copy_(kv_host, non_blocking=True)
+        cg.cg_encode(kvd, codec, kv_dev2, G, 0, T, codes, scales, zeros, None, stream=stream)
+        cg.cg_decode(kvd, codec, codes, scales, zeros, G, 0, T, out, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    e2e_steps = max(2, min(args.steps, 5))
+    with torch.cuda.stream(stream):
+        e2e_step()
+        stream.synchronize()
+        if ws > 1:
+            dist.barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        stream.synchronize()
+    e2e_ms = s0.elapsed_time(s1) / e2e_steps
+
+    # --- max over ranks -----------------------------------------------------------------------
+    vals = torch.tensor([total_ms, statistics.mean(enc_ms), statistics.mean(dec_ms), e2e_ms], dtype=torch.float64,
+                        device=dev)
+    if ws > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, enc_avg, dec_avg, e2e_ms = [float(v) for v in vals.cpu()]
+    if ws > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    ms_step = total_ms / args.steps
+    hbm_peak, peak_kind = _peaks()
+    bpv = 2.0 + args.bits / 8.0 + 4.0 / (16 * G_GROUP)       # algorithmic bytes per value, encode and decode
+    alg_bytes = bpv * n_values
+    enc_gbs = alg_bytes / (enc_avg * 1e-3) / 1e9
+    dec_gbs = alg_bytes / (dec_avg * 1e-3) / 1e9
+    dominant = "cg_encode" if enc_avg >= dec_avg else "cg_decode"
+    dom_ms = max(enc_avg, dec_avg)
+    achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
+    traffic = _traffic_record(dominant, args.bits)
+    value = ws * kv_bytes / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": "KV GB/s for fused gauge+quant encode/decode at %d bits; %% of HBM roofline" % args.bits,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 in/out, fp32 arithmetic, %d-bit codes" % args.bits,
+        "data": "synthetic (seeded AR(1) KV cache, lognormal channel scales, 4 outlier key channels per head)",
+        "config": {"workload": "Llama-3-8B-shaped GQA KV cache 32x2x8x4096x128 bf16, g=16 gauge, block-uniform "
+                               "16x16 ranges, %d bits: encode + decode" % args.bits,
+                   "kv_bytes": kv_bytes, "parallelism": "replicas (dp%d, no collective)" % ws,
+                   "l2": "inputs 0.54 GB > 126 MB L2, no flush"},
+        "encode": {"ms": round(enc_avg, 4), "alg_GBps": round(enc_gbs, 1), "frac": round(enc_gbs / hbm_peak, 4),
+                   "kv_GBps": round(kv_bytes / (enc_avg * 1e-3) / 1e9, 1)},
+        "decode": {"ms": round(dec_avg, 4), "alg_GBps": round(dec_gbs, 1), "frac": round(dec_gbs / hbm_peak, 4),
+                   "kv_GBps": round(kv_bytes / (dec_avg * 1e-3) / 1e9, 1)},
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": hbm_peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "traffic": traffic, "alg_bytes_per_value": bpv},
+        "e2e": {"value": round(ws * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": kv_bytes, "d2h_bytes_per_step": kv_bytes},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.bits, budget_s=args.cpu_seconds)
+    return line
+
+
+def _traffic_record(kernel, bits):
+    """DRAM bytes per launch from the committed ncu summary, if one matches."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        return rec.get("%s_b%d" % (kernel, bits))
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU baseline / reference arm: the oracle, as it stands, on a bounded sample of the workload.
+
+def _oracle_slice_roundtrip(x, G, bits):
+    from oracle import codec as oc
+    enc = oc.encode_block_uniform(x, G, bits)
+    oc.decode_block_uniform(enc["codes"], enc["z"], enc["s"], G, bits)
+
+
+def _oracle_inputs(seed):
+    import numpy as np
+    import torch
+    from oracle import gauge as og
+    from quantization_cg_encode_b200 import synth
+    kv = synth.kv_cache(1, B, 1, T, D, seed=seed, n_outliers=4)      # one (layer, head) of the cache
+    A = synth.gauge_params(1, 1, D // G_GROUP, G_GROUP, sigma=0.1, seed=seed)
+    G = og.gauge_from_A(A.numpy().astype(np.float64)).astype(np.float32).astype(np.float64)
+    return kv.float().numpy().astype(np.float64), G
+
+
+def cpu_baseline(bits, budget_s=15.0):
+    """Oracle encode + decode of whole (layer, head) slices (K and V, 4096 x 128 each)
+    until about budget_s seconds have passed; KV GB/s of what it processed."""
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except Exception:
+        limiter = None
+    x, G = _oracle_inputs(0)
+    n_slice = x.size
+    done, t0 = 0, time.perf_counter()
+    while True:
+        _oracle_slice_roundtrip(x, G, bits)
+        done += 1
+        el = time.perf_counter() - t0
+        if el > budget_s:
+            break
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    gbs = done * 2 * n_slice / el / 1e9
+    return {"value": round(gbs, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d (layer, K+V, head) slices of 2x4096x128 values (%.1f s, numpy fp64/fp32-exact, 1 thread)"
+                      % (done, el)}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return None
+    x, G = _oracle_inputs(0)
+    n_slice = x.size
+    for _ in range(max(0, min(args.warmup, 1))):
+        _oracle_slice_roundtrip(x, G, args.bits)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_slice_roundtrip(x, G, args.bits)
+    el = time.perf_counter() - t0
+    gbs = args.steps * 2 * n_slice / el / 1e9
+    ms = el / args.steps * 1e3
+    line = {
+        "impl": "reference",
+        "metric": "KV GB/s for fused gauge+quant encode/decode at %d bits; %% of HBM roofline" % args.bits,
+        "value": round(gbs, 5), "unit": "GB/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 oracle (fp32-exact codec steps)", "data": "synthetic",
+        "config": {"workload": "Llama-3-8B-shaped GQA KV cache 32x2x8x4096x128 bf16, g=16, 4-bit block-uniform; "
+                               "each step a bounded sample: one (layer, head) K+V slice"},
+        "cpu_baseline": {"value": round(gbs, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "one 2x4096x128 slice per step"},
+        "e2e": {"value": round(gbs, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--bits", type=int, default=4)
+    ap.add_argument("--impl", default="cg", choices=["cg", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "cg":
+        args.warmup = 3
+    line = run_reference(args) if args.impl == "reference" else run_cg(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -14,9 +14,8 @@ namespace cg {
 // (defined once in cg_abi.cu; kernels receive its device address).
 // cg_sync_status() reads and clears it.
 constexpr unsigned int kStatusTimeout = 1u;
-// Upper bound on spins of any mbarrier wait (each spin is a try_wait with the
-// hardware's own suspend hint, so this bounds a wait to well under a second).
-constexpr unsigned int kMaxSpins = 1u << 24;
+// Wall-time bound of any device-side wait on an asynchronous copy.
+constexpr unsigned long long kWaitNs = 2000000000ull;
 
 // ---- problem geometry shared by host and device -------------------------------
 struct KvGeom {
@@ -146,11 +145,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Wait for phase `parity` of `bar` to complete; gives up after kMaxSpins tries,
-// records a timeout in *status and returns false.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for phase `parity` of `bar` to complete.  Gives up after kWaitNs of
+// wall time, ORs kStatusTimeout into *status and returns false (the caller
+// carries on, so every thread still reaches every barrier and the kernel ends).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status) {
-  uint32_t addr = smem_u32(bar);
-  for (unsigned int i = 0; i < kMaxSpins; ++i) {
+  const uint32_t addr = smem_u32(bar);
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
     uint32_t done;
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
@@ -158,9 +164,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
         : "r"(addr), "r"(parity)
         : "memory");
     if (done) return true;
+    if ((i & 255u) == 0) {
+      const uint64_t now = global_ns();
+      if (i == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitNs) {
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
   }
-  atomicOr(status, kStatusTimeout);
-  return false;
 }
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
 // both addresses 16-byte aligned).
@@ -188,6 +201,14 @@ __device__ __forceinline__ void bulk_wait() {
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// 2-D tiled TMA load (no multicast) of box {x, y} into shared memory.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
 }
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -24,6 +24,11 @@ struct CodecArgs {
 };
 
 cudaError_t launch_group_codec(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
+cudaError_t launch_encode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
+
+// 2-D TMA tensor map over a row-major bf16 [rows][cols] array (box_cols x
+// box_rows boxes, 128-byte swizzle); `out` points to a CUtensorMap.
+bool make_tmap_2d_bf16(void* out, const void* base, uint64_t rows, uint64_t cols, int box_cols, int box_rows);
 cudaError_t launch_gauge_build(const float* A, float* G, int n_mats, int g, cudaStream_t st);
 
 }  // namespace cg
