@@ -196,6 +196,10 @@ cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st,
  * a pending CUDA error, else CG_OK. */
 cg_status cg_sync_status(void* stream);
 
+/* Name and description of the CUDA error behind the last CG_ERR_CUDA returned
+ * on the calling host thread ("" if none).  The string is static. */
+const char* cg_last_cuda_error(void);
+
 /* Static, human-readable name of a status code. */
 const char* cg_status_string(cg_status s);
 

@@ -19,7 +19,7 @@ BLOCK_UNIFORM, KIVI = 0, 1
 
 # Every symbol include/cg.h declares.
 EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
-           "cg_spectral_stats", "cg_sync_status", "cg_status_string", "cg_version")
+           "cg_spectral_stats", "cg_sync_status", "cg_last_cuda_error", "cg_status_string", "cg_version")
 
 
 class KvDesc(ctypes.Structure):
@@ -45,7 +45,10 @@ class StatsDesc(ctypes.Structure):
 class CgError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
-        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+        extra = ""
+        if status == CG_ERR_CUDA:
+            extra = ": " + lib().cg_last_cuda_error().decode()
+        super().__init__("%s: %s (status %d)%s" % (where, status_string(status), status, extra))
 
 
 _lib = None
@@ -72,6 +75,7 @@ def lib():
         L.cg_status_string.argtypes = [ctypes.c_int]
         L.cg_status_string.restype = ctypes.c_char_p
         L.cg_version.restype = ctypes.c_int32
+        L.cg_last_cuda_error.restype = ctypes.c_char_p
         for name in ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
                      "cg_spectral_stats", "cg_sync_status"):
             getattr(L, name).restype = ctypes.c_int

@@ -60,7 +60,13 @@ int num_sms() {
 
 KvGeom geom(const cg_kv_desc* kv) { return KvGeom{kv->layers, kv->batch, kv->heads, kv->tokens, kv->d_head}; }
 
-cg_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CG_OK : CG_ERR_CUDA; }
+thread_local cudaError_t t_last_cuda = cudaSuccess;
+
+cg_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return CG_OK;
+  t_last_cuda = e;
+  return CG_ERR_CUDA;
+}
 
 // Device address of the status word on the current device (looked up once
 // per device; a host-side symbol is not a device address).
@@ -130,6 +136,8 @@ cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec, const void
   a.status = status_word();
   if (!a.status) return CG_ERR_CUDA;
   if (a.kivi || a.g == kv->d_head) return CG_ERR_UNSUPPORTED;
+  // g = 16 with an even number of 16-token tiles per head: the specialised kernel
+  if (a.g == 16 && (nt / 16) % 2 == 0) return from_cuda(launch_encode_g16(a, num_sms(), (cudaStream_t)stream));
   return from_cuda(launch_group_codec(a, true, num_sms(), (cudaStream_t)stream));
 }
 
@@ -161,6 +169,7 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec, const uint
   a.status = status_word();
   if (!a.status) return CG_ERR_CUDA;
   if (a.kivi || a.g == kv->d_head) return CG_ERR_UNSUPPORTED;
+  if (a.g == 16) return from_cuda(launch_decode_g16(a, num_sms(), (cudaStream_t)stream));
   return from_cuda(launch_group_codec(a, false, num_sms(), (cudaStream_t)stream));
 }
 
@@ -185,16 +194,21 @@ cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st, const
 
 cg_status cg_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
-  if (e != cudaSuccess) return CG_ERR_CUDA;
+  if (e != cudaSuccess) return from_cuda(e);
   unsigned int flag = 0, zero = 0;
   e = cudaMemcpyFromSymbol(&flag, cg::g_status, sizeof(flag));
-  if (e != cudaSuccess) return CG_ERR_CUDA;
+  if (e != cudaSuccess) return from_cuda(e);
   if (flag) {
     e = cudaMemcpyToSymbol(cg::g_status, &zero, sizeof(zero));
-    if (e != cudaSuccess) return CG_ERR_CUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     return CG_ERR_TIMEOUT;
   }
   return CG_OK;
+}
+
+const char* cg_last_cuda_error(void) {
+  if (t_last_cuda == cudaSuccess) return "";
+  return cudaGetErrorString(t_last_cuda);
 }
 
 const char* cg_status_string(cg_status s) {
