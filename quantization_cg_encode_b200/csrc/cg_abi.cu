@@ -136,8 +136,7 @@ cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec, const void
   a.status = status_word();
   if (!a.status) return CG_ERR_CUDA;
   if (a.kivi || a.g == kv->d_head) return CG_ERR_UNSUPPORTED;
-  // g = 16 with an even number of 16-token tiles per head: the specialised kernel
-  if (a.g == 16 && (nt / 16) % 2 == 0) return from_cuda(launch_encode_g16(a, num_sms(), (cudaStream_t)stream));
+  if (a.g == 16) return from_cuda(launch_encode_g16(a, num_sms(), (cudaStream_t)stream));
   return from_cuda(launch_group_codec(a, true, num_sms(), (cudaStream_t)stream));
 }
 

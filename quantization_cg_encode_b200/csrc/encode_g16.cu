@@ -7,16 +7,20 @@
 //
 // Structure (one CTA per SM, persistent over a contiguous range of 16-token
 // tiles in (layer, K/V, batch, head, token) order, two tiles per iteration):
-//   * tiles (16 tokens x d bf16, 4 KB at d = 128) stream into a 12-stage
-//     shared-memory ring with 2-D TMA loads (128-byte swizzle, no multicast),
-//     completion counted on mbarriers; the warp that releases a stage last
-//     refills it (no producer warp: eight warps of up to 255 registers is what
-//     the 4 x 16K-register scheduler partitions of an SM can hold);
+//   * stages of 4 tiles (64 tokens x d bf16, 16 KB at d = 128) stream into a
+//     6-stage shared-memory ring with 2-D TMA loads of 64 x 64 boxes (8 KB per
+//     copy: smaller copies leave the TMA unit short of HBM bandwidth; 128-byte
+//     swizzle, no multicast), completion counted on mbarriers; the warp that
+//     releases a stage last refills it (no producer warp: eight warps of up to
+//     255 registers is what the 4 x 16K-register scheduler partitions hold);
 //   * warp r owns channel group r: lane (t, hh) = (lane & 15, lane >> 4)
-//     computes gauged outputs 8hh .. 8hh+7 of token t.  Its half of G_r lives
-//     in registers as fp32 row pairs, and the exact per-output FMA chain
-//     (j = 0..15, from +0) runs as packed fma.rn.f32x2, two outputs per
-//     instruction with the token's x_j duplicated into both halves;
+//     computes gauged outputs 8hh .. 8hh+7 of token t in all 4 tiles of a
+//     stage.  Its half of G_r lives in registers as fp32 row pairs, and the
+//     exact per-output FMA chain (j = 0..15, from +0) runs as packed
+//     fma.rn.f32x2, two outputs per instruction with the token's x_j
+//     duplicated into both halves (16 independent chains per thread);
+//   * lanes 8k .. 8k+7 compute tile k's block parameters (one evaluation per
+//     lane covers the stage's four blocks), shared by shuffle;
 //   * the range of a 16 x 16 block is one warp: redux.sync min / max (a
 //     16 x d_head range adds one exchange between the group warps);
 //   * each lane stores its 8 packed codes straight to global memory (a warp
@@ -29,7 +33,7 @@ namespace cg {
 
 namespace {
 
-constexpr int kStages = 12;
+constexpr int kStages = 6;   // ring stages of 4 tiles (96 KB at d = 128)
 
 __device__ __forceinline__ float min3f(float a, float b, float c) {
   float r;
@@ -67,10 +71,11 @@ template <int D, int BITS, bool WFULL>
 struct Cfg {
   static constexpr int NW = D / 16;                      // warps (= channel groups)
   static constexpr int THREADS = NW * 32;
-  static constexpr int TILE_BYTES = 16 * D * 2;          // bf16 input tile
-  static constexpr int BOXES = D / 64;                   // 64-channel TMA boxes per tile
+  static constexpr int TPS = 4;                          // 16-token tiles per ring stage
+  static constexpr int STAGE_BYTES = TPS * 16 * D * 2;   // 16 KB at d = 128: one 8 KB TMA box per 64 channels
+  static constexpr int BOXES = D / 64;
   static constexpr int CODE_TILE = 16 * D * BITS / 8;    // packed codes of one tile
-  static constexpr int SMEM = 1024 + kStages * TILE_BYTES + kStages * 8 + kStages * 4 + 2 * 32 * 4;
+  static constexpr int SMEM = 1024 + kStages * STAGE_BYTES + kStages * 8 + kStages * 4 + 64 * 4;
 };
 
 // Pack 8 codes, given as the bit patterns of (t + 1.5 * 2^23) whose low byte is
@@ -144,36 +149,34 @@ __global__ void __launch_bounds__(Cfg<D, BITS, WFULL>::THREADS, 1)
   constexpr int QMAX = (1 << BITS) - 1;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* stages = base;                                   // kStages x TILE_BYTES, 1024-aligned
-  uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * C::TILE_BYTES);
+  unsigned char* stages = base;                                   // kStages x STAGE_BYTES, 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * C::STAGE_BYTES);
   uint32_t* released = reinterpret_cast<uint32_t*>(full + kStages);
-  float* red = reinterpret_cast<float*>(released + kStages);      // [2 parity][4 (mnA,mxA,mnB,mxB)][8 groups]
+  float* red = reinterpret_cast<float*>(released + kStages);      // [min / max][4 tiles][8 groups]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Work unit = a pair of consecutive tiles of one head slice (the tile count
-  // per slice is even on this path); the CTA owns tiles [2 u0, 2 u1).
-  const int tps = a.nt / 16;
-  const int upt = tps / 2;
-  const long long total = (long long)upt * a.k.slices();
+  // Work unit = one ring stage: up to 4 consecutive tiles of one head slice,
+  // processed as two pairs (A, B).  The CTA owns units [u0, u1).
+  const int tps = a.nt / 16;                                      // tiles per head slice
+  const int sps = (tps + C::TPS - 1) / C::TPS;                    // stages per head slice
+  const long long total = (long long)sps * a.k.slices();
   const long long u0 = total * blockIdx.x / gridDim.x;
   const long long u1 = total * (blockIdx.x + 1) / gridDim.x;
   const int n_units = (int)(u1 - u0);
-  const int n_tiles = 2 * n_units;
-  long long slice = u0 / upt;
-  int pu = (int)(u0 - slice * upt);                               // pair index inside the slice
 
-  // row of the CTA's j-th tile in the [rows][d] view of the cache
-  auto tile_row = [&](int j) -> int {
-    const unsigned gt = (unsigned)(2 * u0 + j);   // < 2^31 tiles
-    const unsigned sl = gt / (unsigned)tps;
-    return (int)((long long)sl * a.k.T + a.t0 + 16 * (gt - sl * (unsigned)tps));
+  // rows [row, row + 64) of the [rows][d] view hold unit q's tiles
+  auto unit_row = [&](int q) -> int {
+    const unsigned gu = (unsigned)(u0 + q);                       // < 2^31 units
+    const unsigned sl = gu / (unsigned)sps;
+    return (int)((long long)sl * a.k.T + a.t0 + 64 * (gu - sl * (unsigned)sps));
   };
-  auto issue = [&](int j) {
-    const int st = j % kStages;
-    mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
-    const int row = tile_row(j);
+  auto issue = [&](int q) {
+    const int st = q % kStages;
+    mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+    const int row = unit_row(q);
 #pragma unroll
-    for (int b = 0; b < C::BOXES; ++b) tma_load_2d(stages + st * C::TILE_BYTES + b * 2048, &tmap, b * 64, row, &full[st]);
+    for (int b = 0; b < C::BOXES; ++b)
+      tma_load_2d(stages + st * C::STAGE_BYTES + b * (C::STAGE_BYTES / C::BOXES), &tmap, b * 64, row, &full[st]);
   };
 
   if (threadIdx.x == 0) {
@@ -182,150 +185,162 @@ __global__ void __launch_bounds__(Cfg<D, BITS, WFULL>::THREADS, 1)
       released[s] = 0;
     }
     fence_mbar_init();
-    for (int j = 0; j < kStages && j < n_tiles; ++j) issue(j);
+    for (int q = 0; q < kStages && q < n_units; ++q) issue(q);
   }
   __syncthreads();
+  if (n_units == 0) return;
 
-  // ---------------- consumers: warp r = channel group r ----------------
   const int r = warp;
   const int t = lane & 15, hh = lane >> 4;
   const double inv_qmax = 1.0 / (double)QMAX;
   const int box = r >> 2;
   const int c0 = (r & 3) * 2;  // first 16-byte chunk of this group inside the 128-byte row
-  const uint32_t rd0 = t * 128 + ((c0 ^ (t & 7)) << 4) + box * 2048;
-  const uint32_t rd1 = t * 128 + (((c0 + 1) ^ (t & 7)) << 4) + box * 2048;
+  // byte offsets of token t's two chunks inside the first tile of a stage (box rows t)
+  const uint32_t rd0 = box * (C::STAGE_BYTES / C::BOXES) + t * 128 + ((c0 ^ (t & 7)) << 4);
+  const uint32_t rd1 = box * (C::STAGE_BYTES / C::BOXES) + t * 128 + (((c0 + 1) ^ (t & 7)) << 4);
   const int nblk = WFULL ? 1 : D / 16;
   const int code_off = WFULL ? (t * D + 16 * r + 8 * hh) * BITS / 8 : r * (256 * BITS / 8) + t * (2 * BITS) + hh * BITS;
   const long long slice_code_bytes = (long long)a.k.T * D * BITS / 8;
   const long long slice_blocks = (long long)(a.k.T / 16) * nblk;
 
   f2_t gp[4][16];  // gp[m][j] = {G[8hh+2m][j], G[8hh+2m+1][j]}
-  bool need_g = true;
-  for (int u = 0; u < n_units; ++u) {
-    if (need_g) {
-      int l, sk, b, h;
-      slice_coords(slice, a.k, l, sk, b, h);
-      const float* Gr = a.G + (gauge_set(l, sk, h, a.k) * (D / 16) + r) * 256;
+  auto load_g = [&](long long sl) {
+    int l, sk, b, h;
+    slice_coords(sl, a.k, l, sk, b, h);
+    const float* Gr = a.G + (gauge_set(l, sk, h, a.k) * (D / 16) + r) * 256;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float4* row0 = reinterpret_cast<const float4*>(Gr + (8 * hh + 2 * m) * 16);
-        const float4* row1 = reinterpret_cast<const float4*>(Gr + (8 * hh + 2 * m + 1) * 16);
+    for (int m = 0; m < 4; ++m) {
+      const float4* row0 = reinterpret_cast<const float4*>(Gr + (8 * hh + 2 * m) * 16);
+      const float4* row1 = reinterpret_cast<const float4*>(Gr + (8 * hh + 2 * m + 1) * 16);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 uu = __ldg(row0 + q), vv = __ldg(row1 + q);
-          gp[m][4 * q + 0] = f2_make(uu.x, vv.x);
-          gp[m][4 * q + 1] = f2_make(uu.y, vv.y);
-          gp[m][4 * q + 2] = f2_make(uu.z, vv.z);
-          gp[m][4 * q + 3] = f2_make(uu.w, vv.w);
-        }
+      for (int q = 0; q < 4; ++q) {
+        const float4 uu = __ldg(row0 + q), vv = __ldg(row1 + q);
+        gp[m][4 * q + 0] = f2_make(uu.x, vv.x);
+        gp[m][4 * q + 1] = f2_make(uu.y, vv.y);
+        gp[m][4 * q + 2] = f2_make(uu.z, vv.z);
+        gp[m][4 * q + 3] = f2_make(uu.w, vv.w);
       }
-      need_g = false;
     }
-    const int tileA = a.t0 / 16 + 2 * pu;
-
-    // ---- x of token t in group r, tiles A = 2u and B = 2u + 1 of this CTA ----
-    const int jA = 2 * u, jB = 2 * u + 1;
-    const int sA = jA % kStages, sB = jB % kStages;
-    mbar_wait(&full[sA], (uint32_t)((jA / kStages) & 1), a.status);
-    const uint4 a0 = *reinterpret_cast<const uint4*>(stages + sA * C::TILE_BYTES + rd0);
-    const uint4 a1 = *reinterpret_cast<const uint4*>(stages + sA * C::TILE_BYTES + rd1);
-    mbar_wait(&full[sB], (uint32_t)((jB / kStages) & 1), a.status);
-    const uint4 b0 = *reinterpret_cast<const uint4*>(stages + sB * C::TILE_BYTES + rd0);
-    const uint4 b1 = *reinterpret_cast<const uint4*>(stages + sB * C::TILE_BYTES + rd1);
+  };
+  // the warp is done reading unit q; the last warp to say so refills the stage
+  auto release = [&](int q) {
     __syncwarp();
     if (lane == 0) {
-      if (stage_release(&released[sA]) == C::NW - 1) {
-        released[sA] = 0;
-        if (jA + kStages < n_tiles) issue(jA + kStages);
-      }
-      if (stage_release(&released[sB]) == C::NW - 1) {
-        released[sB] = 0;
-        if (jB + kStages < n_tiles) issue(jB + kStages);
+      const int st = q % kStages;
+      if (stage_release(&released[st]) == C::NW - 1) {
+        released[st] = 0;
+        if (q + kStages < n_units) issue(q + kStages);
       }
     }
+  };
 
-    // ---- gauge: exact fp32 FMA chains, tiles A and B interleaved ----
-    const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-    const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-    f2_t accA[4], accB[4];
+  // One iteration = one stage of up to 4 tiles: 16 independent FMA chains per
+  // thread, then the four blocks' parameters computed by 8 lanes each.
+  long long slice = u0 / sps;
+  int sq = (int)(u0 - slice * sps);
+  load_g(slice);
+  const int kq = lane >> 3;  // tile whose block parameters this lane computes
+  for (int q = 0; q < n_units; ++q) {
+    const int nvalid = min(C::TPS, tps - C::TPS * sq);
+    const int st = q % kStages;
+    mbar_wait(&full[st], (uint32_t)(q / kStages) & 1u, a.status);
+    const unsigned char* sb = stages + st * C::STAGE_BYTES;
+    uint32_t w[C::TPS][8];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) accA[m] = accB[m] = 0ull;  // {+0, +0}
+    for (int k = 0; k < C::TPS; ++k) {
+      const uint4 v0 = *reinterpret_cast<const uint4*>(sb + k * 2048 + rd0);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(sb + k * 2048 + rd1);
+      w[k][0] = v0.x; w[k][1] = v0.y; w[k][2] = v0.z; w[k][3] = v0.w;
+      w[k][4] = v1.x; w[k][5] = v1.y; w[k][6] = v1.z; w[k][7] = v1.w;
+    }
+    // ---- gauge: exact fp32 FMA chains (j = 0..15 from +0), four tiles interleaved ----
+    f2_t acc[C::TPS][4];
+#pragma unroll
+    for (int k = 0; k < C::TPS; ++k)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[k][m] = 0ull;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const float xa = (j & 1) ? bf16hi(wa[j >> 1]) : bf16lo(wa[j >> 1]);
-      const float xb = (j & 1) ? bf16hi(wb[j >> 1]) : bf16lo(wb[j >> 1]);
-      const f2_t xda = f2_make(xa, xa), xdb = f2_make(xb, xb);
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        accA[m] = f2_fma(gp[m][j], xda, accA[m]);
-        accB[m] = f2_fma(gp[m][j], xdb, accB[m]);
+      for (int k = 0; k < C::TPS; ++k) {
+        const float x = (j & 1) ? bf16hi(w[k][j >> 1]) : bf16lo(w[k][j >> 1]);
+        const f2_t xd = f2_make(x, x);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) acc[k][m] = f2_fma(gp[m][j], xd, acc[k][m]);
       }
     }
-    if (a.gauged) {
-      float* gA = a.gauged + (slice * a.k.T + (long long)tileA * 16 + t) * D + 16 * r + 8 * hh;
-      float y[8];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) f2_split(accA[m], y[2 * m], y[2 * m + 1]);
-      reinterpret_cast<float4*>(gA)[0] = make_float4(y[0], y[1], y[2], y[3]);
-      reinterpret_cast<float4*>(gA)[1] = make_float4(y[4], y[5], y[6], y[7]);
-      {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) f2_split(accB[m], y[2 * m], y[2 * m + 1]);
-        reinterpret_cast<float4*>(gA + 16 * D)[0] = make_float4(y[0], y[1], y[2], y[3]);
-        reinterpret_cast<float4*>(gA + 16 * D)[1] = make_float4(y[4], y[5], y[6], y[7]);
-      }
-    }
+    release(q);
 
     // ---- block ranges ----
-    float mnA, mxA, mnB, mxB;
-    minmax8(accA, mnA, mxA);
-    minmax8(accB, mnB, mxB);
-    mnA = warp_min_f32(mnA);
-    mxA = warp_max_f32(mxA);
-    mnB = warp_min_f32(mnB);
-    mxB = warp_max_f32(mxB);
+    float mn[C::TPS], mx[C::TPS];
+#pragma unroll
+    for (int k = 0; k < C::TPS; ++k) {
+      minmax8(acc[k], mn[k], mx[k]);
+      mn[k] = warp_min_f32(mn[k]);
+      mx[k] = warp_max_f32(mx[k]);
+    }
     if constexpr (WFULL) {
-      float* rb = red + (u & 1) * 32;
+      float* rb = red;  // [mn x 4 tiles][mx x 4 tiles] x 8 groups
       if (lane == 0) {
-        rb[r] = mnA;
-        rb[8 + r] = mxA;
-        rb[16 + r] = mnB;
-        rb[24 + r] = mxB;
+#pragma unroll
+        for (int k = 0; k < C::TPS; ++k) {
+          rb[k * 8 + r] = mn[k];
+          rb[32 + k * 8 + r] = mx[k];
+        }
       }
       named_bar_sync(1, C::NW * 32);
-      mnA = rb[0]; mxA = rb[8]; mnB = rb[16]; mxB = rb[24];
 #pragma unroll
-      for (int q = 1; q < C::NW; ++q) {
-        mnA = fminf(mnA, rb[q]);
-        mxA = fmaxf(mxA, rb[8 + q]);
-        mnB = fminf(mnB, rb[16 + q]);
-        mxB = fmaxf(mxB, rb[24 + q]);
+      for (int k = 0; k < C::TPS; ++k) {
+        mn[k] = rb[k * 8];
+        mx[k] = rb[32 + k * 8];
+#pragma unroll
+        for (int g = 1; g < C::NW; ++g) {
+          mn[k] = fminf(mn[k], rb[k * 8 + g]);
+          mx[k] = fmaxf(mx[k], rb[32 + k * 8 + g]);
+        }
       }
+      named_bar_sync(2, C::NW * 32);  // every warp has read rb before it is reused
     }
-    // block parameters: lanes 0-15 for tile A, lanes 16-31 for tile B
-    const float pmn = hh ? mnB : mnA, pmx = hh ? mxB : mxA;
+    // ---- block parameters: lanes 8k .. 8k+7 compute tile k's ----
+    const float pmn = kq == 0 ? mn[0] : kq == 1 ? mn[1] : kq == 2 ? mn[2] : mn[3];
+    const float pmx = kq == 0 ? mx[0] : kq == 1 ? mx[1] : kq == 2 ? mx[2] : mx[3];
     const QParams qp = quant_params(pmn, pmx, inv_qmax);
     const float tlo = __fmul_rn(__fsub_rn(pmn, qp.zf), qp.inv);
     const float thi = __fmul_rn(__fsub_rn(pmx, qp.zf), qp.inv);
     // t is monotone in y: if the block's extremes round into [0, qmax], no value needs clamping
     const unsigned inr = __ballot_sync(0xffffffffu, (tlo >= -0.5f) && (thi < (float)QMAX + 0.5f));
-    const float zfA = __shfl_sync(0xffffffffu, qp.zf, 0), invA = __shfl_sync(0xffffffffu, qp.inv, 0);
-    const float zfB = __shfl_sync(0xffffffffu, qp.zf, 16), invB = __shfl_sync(0xffffffffu, qp.inv, 16);
 
-    const uint64_t chA = quantize8<BITS>(accA, zfA, invA, inr & 1u);
-    const uint64_t chB = quantize8<BITS>(accB, zfB, invB, (inr >> 16) & 1u);
-    uint8_t* cp = a.codes + slice * slice_code_bytes + (long long)tileA * C::CODE_TILE + code_off;
-    store_chunk<BITS>(cp, chA);
-    store_chunk<BITS>(cp + C::CODE_TILE, chB);
-    if ((lane & 15) == 0 && (!WFULL || r == 0)) {
-      const long long bidx = slice * slice_blocks + (long long)(tileA + hh) * nblk + (WFULL ? 0 : r);
+    // ---- quantize, pack, store ----
+    const int tile0 = a.t0 / 16 + C::TPS * sq;
+    uint8_t* cp = a.codes + slice * slice_code_bytes + (long long)tile0 * C::CODE_TILE + code_off;
+#pragma unroll
+    for (int k = 0; k < C::TPS; ++k) {
+      const float zf = __shfl_sync(0xffffffffu, qp.zf, 8 * k);
+      const float inv = __shfl_sync(0xffffffffu, qp.inv, 8 * k);
+      const uint64_t ch = quantize8<BITS>(acc[k], zf, inv, (inr >> (8 * k)) & 1u);
+      if (k < nvalid) store_chunk<BITS>(cp + k * C::CODE_TILE, ch);
+    }
+    if ((lane & 7) == 0 && kq < nvalid && (!WFULL || r == 0)) {
+      const long long bidx = slice * slice_blocks + (long long)(tile0 + kq) * nblk + (WFULL ? 0 : r);
       a.scales[bidx] = qp.sh;
       a.zeros[bidx] = qp.zh;
     }
-    if (++pu == upt) {
-      pu = 0;
+    if (a.gauged) {
+#pragma unroll
+      for (int k = 0; k < C::TPS; ++k) {
+        if (k >= nvalid) break;
+        float* gk = a.gauged + (slice * a.k.T + (long long)(tile0 + k) * 16 + t) * D + 16 * r + 8 * hh;
+        float y[8];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) f2_split(acc[k][m], y[2 * m], y[2 * m + 1]);
+        reinterpret_cast<float4*>(gk)[0] = make_float4(y[0], y[1], y[2], y[3]);
+        reinterpret_cast<float4*>(gk)[1] = make_float4(y[4], y[5], y[6], y[7]);
+      }
+    }
+    if (++sq == sps) {
+      sq = 0;
       ++slice;
-      need_g = true;
+      if (q + 1 < n_units) load_g(slice);
     }
   }
 }
@@ -335,11 +350,11 @@ cudaError_t launch_one(const CodecArgs& a, int num_sms, cudaStream_t st) {
   using C = Cfg<D, BITS, WFULL>;
   alignas(64) CUtensorMap tmap;
   const uint64_t rows = (uint64_t)a.k.slices() * a.k.T;
-  if (!make_tmap_2d_bf16(&tmap, a.kv, rows, D, 64, 16)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d_bf16(&tmap, a.kv, rows, D, 64, 16 * C::TPS)) return cudaErrorInvalidValue;
   auto kern = encode_g16_kernel<D, BITS, WFULL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  const long long total = (long long)(a.nt / 32) * a.k.slices();
+  const long long total = (long long)((a.nt / 16 + C::TPS - 1) / C::TPS) * a.k.slices();
   const int grid = (int)(total < num_sms ? total : num_sms);
   kern<<<grid, C::THREADS, C::SMEM, st>>>(tmap, a);
   return cudaGetLastError();
@@ -366,7 +381,6 @@ cudaError_t launch_b(const CodecArgs& a, int num_sms, cudaStream_t st) {
 
 cudaError_t launch_encode_g16(const CodecArgs& a, int num_sms, cudaStream_t st) {
   if (a.nt == 0) return cudaSuccess;
-  if ((a.nt / 16) % 2 != 0) return cudaErrorInvalidValue;   // callers route odd tile counts elsewhere
   return a.k.d == 128 ? launch_b<128>(a, num_sms, st) : launch_b<64>(a, num_sms, st);
 }
 
