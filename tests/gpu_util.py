@@ -68,3 +68,18 @@ def assert_close_bf16(got, ref, rel_norm=2e-3, what=""):
     bad = np.abs(flat_g - flat_r) > bound
     assert not bad.any(), "%s: %d elements beyond the bf16 bound, worst %.3g" % (
         what, int(bad.sum()), float((np.abs(flat_g - flat_r) - bound).max()))
+
+
+def kivi_np(codes, scales, zeros, shape, bits):
+    """Device KIVI buffers -> (keys, values) numpy views matching the oracle's layout."""
+    L, _, B, H, T, d = shape
+    per = T * d * bits // 8
+    c = codes.cpu().numpy().reshape(L, 2, B, H, per)
+    nr = T * d // 32
+    s = fp16_bits(scales).reshape(L, 2, B, H, nr)
+    z = fp16_bits(zeros).reshape(L, 2, B, H, nr)
+    keys = dict(codes=c[:, 0].reshape(L, B, H, T // 32, d, 4 * bits), s=s[:, 0].reshape(L, B, H, T // 32, d),
+                z=z[:, 0].reshape(L, B, H, T // 32, d))
+    vals = dict(codes=c[:, 1].reshape(L, B, H, T, d // 32, 4 * bits), s=s[:, 1].reshape(L, B, H, T, d // 32),
+                z=z[:, 1].reshape(L, B, H, T, d // 32))
+    return keys, vals
