@@ -136,7 +136,10 @@ cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec, const void
   a.status = status_word();
   if (!a.status) return CG_ERR_CUDA;
   if (a.kivi) return from_cuda(launch_kivi(a, true, num_sms(), (cudaStream_t)stream));
-  if (a.g == kv->d_head) return CG_ERR_UNSUPPORTED;
+  if (a.g == kv->d_head) {
+    if (kv->d_head != 128) return CG_ERR_UNSUPPORTED;
+    return from_cuda(launch_fullhead(a, true, num_sms(), (cudaStream_t)stream));
+  }
   if (a.g == 16) return from_cuda(launch_encode_g16(a, num_sms(), (cudaStream_t)stream));
   return from_cuda(launch_group_codec(a, true, num_sms(), (cudaStream_t)stream));
 }
@@ -169,7 +172,10 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec, const uint
   a.status = status_word();
   if (!a.status) return CG_ERR_CUDA;
   if (a.kivi) return from_cuda(launch_kivi(a, false, num_sms(), (cudaStream_t)stream));
-  if (a.g == kv->d_head) return CG_ERR_UNSUPPORTED;
+  if (a.g == kv->d_head) {
+    if (kv->d_head != 128) return CG_ERR_UNSUPPORTED;
+    return from_cuda(launch_fullhead(a, false, num_sms(), (cudaStream_t)stream));
+  }
   if (a.g == 16) return from_cuda(launch_decode_g16(a, num_sms(), (cudaStream_t)stream));
   return from_cuda(launch_group_codec(a, false, num_sms(), (cudaStream_t)stream));
 }

@@ -27,6 +27,7 @@ cudaError_t launch_group_codec(const CodecArgs& a, bool encode, int num_sms, cud
 cudaError_t launch_encode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_decode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_kivi(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
+cudaError_t launch_fullhead(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
 
 // 2-D TMA tensor map over a row-major bf16 [rows][cols] array (box_cols x
 // box_rows boxes, 128-byte swizzle); `out` points to a CUtensorMap.

@@ -1,0 +1,605 @@
+// Full-head gauge (g = d_head = 128): the gauge is a dense 128 x 128
+// contraction per token, run on the 5th-generation tensor cores.
+//
+// Codec-Gauge, Method: full-head gauges (g = d_l) give the gauge the most
+// freedom; explicit application costs O(N_KV g) multiply-adds (128 per value
+// here), and recovery before attention is explicit.  Experimental setup:
+// block-uniform backend; with g = d_head a range block is 16 tokens x d_head.
+//
+// Encode, per block of 128 tokens of one head slice:
+//   * a TMA warp streams x blocks (128 x 128 bf16 = 32 KB, two 16 KB boxes with
+//     128-byte swizzle, no multicast) into a 3-stage shared-memory ring, and
+//     writes each head slice's G as bf16 (RNE) in the same swizzled K-major
+//     layout (two buffers, so the next slice's G is staged while the current
+//     one is in use);
+//   * one thread issues 8 tcgen05.mma (M = N = 128, K = 16, bf16 x bf16 -> fp32)
+//     into one of two 128-column TMEM accumulators: y[t][i] = sum_j x[t][j] G[i][j];
+//   * four epilogue warps (one thread per token) read their row with
+//     tcgen05.ld, reduce the 16-token ranges with half-warp shuffles and
+//     quantize, pack and store exactly like the grouped encoder.
+// Every wait on an mbarrier is bounded in time.
+#include <cuda.h>
+
+#include "cg_kernels.cuh"
+
+namespace cg {
+
+namespace {
+
+constexpr int kXStages = 3;
+constexpr int kBlockBytes = 128 * 128 * 2;  // 32 KB of bf16
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = (kEpiWarps + 2) * 32;  // 4 epilogue, 1 TMA / G, 1 MMA
+// tcgen05 instruction descriptor: D fp32, A and B bf16, both K-major, N = 128, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+// Shared-memory matrix descriptor for a K-major tile in the 128-byte swizzled
+// canonical layout (rows of 128 bytes, 8-row atoms 1024 bytes apart).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);  // start address
+  d |= (uint64_t)1 << 16;                         // leading byte offset (unused for swizzled K-major): 16 B
+  d |= (uint64_t)(1024 >> 4) << 32;               // stride byte offset: 1024 B between 8-row groups
+  d |= (uint64_t)1 << 46;                         // descriptor version
+  d |= (uint64_t)2 << 61;                         // layout: 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Byte offset of element (row, col) of a 128 x 128 bf16 K-major tile stored
+// as two 64-column halves in the 128-byte swizzled layout.
+__device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
+  const int half = col >> 6, c = (col & 63) >> 3;
+  return half * 16384 + row * 128 + ((c ^ (row & 7)) << 4) + (col & 7) * 2;
+}
+
+struct FhSmem {
+  unsigned char* xs;  // kXStages x 32 KB, 1024-aligned
+  unsigned char* gs;  // 2 x 32 KB
+  uint64_t* x_full;
+  uint64_t* x_empty;
+  uint64_t* g_full;
+  uint64_t* g_empty;
+  uint64_t* t_full;
+  uint64_t* t_empty;
+  uint32_t* tmem_base;
+};
+
+__device__ inline FhSmem fh_carve(unsigned char* raw) {
+  FhSmem s;
+  unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)raw + 1023) & ~(uintptr_t)1023);
+  s.xs = base;
+  s.gs = base + kXStages * kBlockBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.gs + 2 * kBlockBytes);
+  s.x_full = bars;
+  s.x_empty = bars + kXStages;
+  s.g_full = bars + 2 * kXStages;
+  s.g_empty = s.g_full + 2;
+  s.t_full = s.g_empty + 2;
+  s.t_empty = s.t_full + 2;
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.t_empty + 2);
+  return s;
+}
+constexpr int kFhSmem = 1024 + (kXStages + 2) * kBlockBytes + (2 * kXStages + 6) * 8 + 16;
+
+}  // namespace
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+    fullhead_encode_kernel(const __grid_constant__ CUtensorMap tmap, CodecArgs a) {
+  constexpr int D = 128;
+  constexpr int QMAX = (1 << BITS) - 1;
+  extern __shared__ unsigned char smem_raw[];
+  const FhSmem sm = fh_carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bps = (a.nt + 127) / 128;  // 128-token blocks per head slice
+  const long long total = (long long)bps * a.k.slices();
+  const long long b0 = total * blockIdx.x / gridDim.x;
+  const long long b1 = total * (blockIdx.x + 1) / gridDim.x;
+  const int n_blocks = (int)(b1 - b0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kXStages; ++s) {
+      mbar_init(&sm.x_full[s], 1);
+      mbar_init(&sm.x_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.g_full[s], 1);
+      mbar_init(&sm.g_empty[s], 1);
+      mbar_init(&sm.t_full[s], 1);
+      mbar_init(&sm.t_empty[s], kEpiWarps);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0) {  // TMEM: two 128-column fp32 accumulators
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(sm.tmem_base)),
+                 "r"(256));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sm.tmem_base;
+
+  if (warp == kEpiWarps) {
+    // ---------------- TMA x blocks + G staging ----------------
+    long long slice = b0 / bps;
+    int bq = (int)(b0 - slice * bps);
+    int gcount = 0;  // slices staged so far
+    for (int i = 0; i < n_blocks; ++i) {
+      if (i == 0 || bq == 0) {  // new head slice: stage its G (bf16, swizzled K-major, rows = outputs)
+        const int gb = gcount & 1;
+        mbar_wait(&sm.g_empty[gb], ((uint32_t)(gcount >> 1) & 1u) ^ 1u, a.status);
+        int l, sk, b, h;
+        slice_coords(slice, a.k, l, sk, b, h);
+        const float4* Gp = reinterpret_cast<const float4*>(a.G + gauge_set(l, sk, h, a.k) * D * D);
+        unsigned char* gdst = sm.gs + gb * kBlockBytes;
+        for (int e = lane; e < D * D / 8; e += 32) {  // 8 consecutive elements of one row per step
+          const float4 u = __ldg(Gp + 2 * e), v = __ldg(Gp + 2 * e + 1);
+          const int row = (e * 8) / D, col = (e * 8) % D;
+          uint4 w;
+          w.x = pack_bf16x2(u.x, u.y);
+          w.y = pack_bf16x2(u.z, u.w);
+          w.z = pack_bf16x2(v.x, v.y);
+          w.w = pack_bf16x2(v.z, v.w);
+          *reinterpret_cast<uint4*>(gdst + sw128_offset(row, col)) = w;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.g_full[gb]);
+        ++gcount;
+      }
+      if (lane == 0) {
+        const int s = i % kXStages;
+        mbar_wait(&sm.x_empty[s], ((uint32_t)(i / kXStages) & 1u) ^ 1u, a.status);
+        mbar_arrive_expect_tx(&sm.x_full[s], kBlockBytes);
+        const int row0 = (int)(slice * a.k.T + a.t0 + 128LL * bq);
+        tma_load_2d(sm.xs + s * kBlockBytes, &tmap, 0, row0, &sm.x_full[s]);
+        tma_load_2d(sm.xs + s * kBlockBytes + 16384, &tmap, 64, row0, &sm.x_full[s]);
+      }
+      __syncwarp();
+      if (++bq == bps) {
+        bq = 0;
+        ++slice;
+      }
+    }
+  } else if (warp == kEpiWarps + 1) {
+    // ---------------- MMA issue (one thread) ----------------
+    if (lane == 0) {
+      long long slice = b0 / bps;
+      int bq = (int)(b0 - slice * bps);
+      int gcount = 0;
+      for (int i = 0; i < n_blocks; ++i) {
+        const int gb = gcount & 1;
+        if (i == 0 || bq == 0) mbar_wait(&sm.g_full[gb], (uint32_t)(gcount >> 1) & 1u, a.status);
+        const int s = i % kXStages, acc = i & 1;
+        mbar_wait(&sm.x_full[s], (uint32_t)(i / kXStages) & 1u, a.status);
+        mbar_wait(&sm.t_empty[acc], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.status);
+        tc_fence_after();
+        const uint32_t xa = smem_u32(sm.xs + s * kBlockBytes), ga = smem_u32(sm.gs + gb * kBlockBytes);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t koff = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_bf16(tmem + acc * 128, sw128_desc(xa + koff), sw128_desc(ga + koff), k > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.x_empty[s]);
+        umma_commit(&sm.t_full[acc]);
+        const bool last_of_slice = (bq + 1 == bps) || (i + 1 == n_blocks);
+        if (last_of_slice) {
+          umma_commit(&sm.g_empty[gb]);
+          ++gcount;
+        }
+        if (++bq == bps) {
+          bq = 0;
+          ++slice;
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: thread = token row of the block ----------------
+    const int row = 32 * warp + lane;
+    const double inv_qmax = 1.0 / (double)QMAX;
+    const long long slice_code_bytes = (long long)a.k.T * D * BITS / 8;
+    long long slice = b0 / bps;
+    int bq = (int)(b0 - slice * bps);
+    for (int i = 0; i < n_blocks; ++i) {
+      const int acc = i & 1;
+      mbar_wait(&sm.t_full[acc], (uint32_t)(i >> 1) & 1u, a.status);
+      tc_fence_after();
+      float y[128];
+      const uint32_t taddr = tmem + acc * 128 + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(taddr + 32 * c, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[32 * c + j] = v[j];
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.t_empty[acc]);
+
+      const int valid = min(128, a.nt - 128 * bq);
+      const int tok = a.t0 + 128 * bq + row;
+      // range of the 16-token block: this row's 128 values, then 16 lanes
+      float mn = y[0], mx = y[0];
+#pragma unroll
+      for (int j = 1; j < 128; ++j) {
+        mn = fminf(mn, y[j]);
+        mx = fmaxf(mx, y[j]);
+      }
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (row < valid) {
+        const QParams qp = quant_params(mn, mx, inv_qmax);
+        if (a.gauged) {
+          float4* gd = reinterpret_cast<float4*>(a.gauged + (slice * a.k.T + tok) * D);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) gd[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+        }
+        // token row's 128 codes: bytes [r16 * 16 * BITS, +16 * BITS) of its block's record
+        uint32_t words[4 * BITS];
+#pragma unroll
+        for (int w = 0; w < 4 * BITS; ++w) words[w] = 0;
+#pragma unroll
+        for (int j = 0; j < 128; ++j) {
+          const uint32_t q = quantize_one(y[j], qp.zf, qp.inv, QMAX);
+          const int bit = j * BITS;
+          words[bit >> 5] |= q << (bit & 31);
+          if ((bit & 31) + BITS > 32) words[(bit >> 5) + 1] |= q >> (32 - (bit & 31));
+        }
+        const int tile = tok / 16, r16 = tok % 16;
+        uint4* dst = reinterpret_cast<uint4*>(a.codes + slice * slice_code_bytes + (long long)tile * (16 * D * BITS / 8) +
+                                              r16 * (D * BITS / 8));
+#pragma unroll
+        for (int w = 0; w < BITS; ++w) dst[w] = make_uint4(words[4 * w], words[4 * w + 1], words[4 * w + 2], words[4 * w + 3]);
+        if ((lane & 15) == 0) {
+          const long long bidx = slice * (a.k.T / 16) + tile;
+          a.scales[bidx] = qp.sh;
+          a.zeros[bidx] = qp.zh;
+        }
+      }
+      if (++bq == bps) {
+        bq = 0;
+        ++slice;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+  }
+}
+
+
+// Decode, per block of 128 tokens: x_hat_t = G^T (s q_t + z) = s (G^T q_t) + z (G^T 1)
+// (the range block of 16 tokens x d_head has one s and z).  Four warps expand
+// the codes into the A operand (exact bf16 integers, swizzled K-major rows in
+// shared memory) for block i+1 while the tensor cores contract block i with
+// B = G^T (bf16, swizzled K-major, column sums of the same bf16 values kept
+// beside it); the same warps then read the accumulator and write bf16.
+namespace {
+constexpr int kDecThreads = (kEpiWarps + 2) * 32;
+struct FdSmem {
+  unsigned char* as;  // 2 x 32 KB A tiles
+  unsigned char* gs;  // 2 x 32 KB G^T tiles
+  float* colsum;      // 2 x 128
+  uint64_t* a_full;
+  uint64_t* a_empty;
+  uint64_t* g_full;
+  uint64_t* g_empty;
+  uint64_t* t_full;
+  uint64_t* t_empty;
+  uint32_t* tmem_base;
+};
+__device__ inline FdSmem fd_carve(unsigned char* raw) {
+  FdSmem s;
+  unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)raw + 1023) & ~(uintptr_t)1023);
+  s.as = base;
+  s.gs = base + 2 * kBlockBytes;
+  s.colsum = reinterpret_cast<float*>(base + 4 * kBlockBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.colsum + 256);
+  s.a_full = bars;
+  s.a_empty = bars + 2;
+  s.g_full = bars + 4;
+  s.g_empty = bars + 6;
+  s.t_full = bars + 8;
+  s.t_empty = bars + 10;
+  s.tmem_base = reinterpret_cast<uint32_t*>(bars + 12);
+  return s;
+}
+constexpr int kFdSmem = 1024 + 4 * kBlockBytes + 256 * 4 + 12 * 8 + 16;
+
+// bf16 bits of two codes (< 256, exact), packed low / high
+__device__ __forceinline__ uint32_t code_pair_bf16(uint32_t q0, uint32_t q1) {
+  const f2_t v = f2_add(f2_make(__uint_as_float(0x4B000000u | q0), __uint_as_float(0x4B000000u | q1)),
+                        f2_make(-8388608.0f, -8388608.0f));
+  float lo, hi;
+  f2_split(v, lo, hi);
+  return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
+}
+}  // namespace
+
+template <int BITS>
+__global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecArgs a) {
+  constexpr int D = 128;
+  constexpr uint32_t M = (1u << BITS) - 1u;
+  extern __shared__ unsigned char smem_raw[];
+  const FdSmem sm = fd_carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bps = (a.nt + 127) / 128;
+  const long long total = (long long)bps * a.k.slices();
+  const long long b0 = total * blockIdx.x / gridDim.x;
+  const long long b1 = total * (blockIdx.x + 1) / gridDim.x;
+  const int n_blocks = (int)(b1 - b0);
+  const long long slice_code_bytes = (long long)a.k.T * D * BITS / 8;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.a_full[s], kEpiWarps);
+      mbar_init(&sm.a_empty[s], 1);
+      mbar_init(&sm.g_full[s], 1);
+      // released by the tensor cores (done reading G^T) and by the epilogue
+      // warps (done reading the column sums)
+      mbar_init(&sm.g_empty[s], 1 + kEpiWarps);
+      mbar_init(&sm.t_full[s], 1);
+      mbar_init(&sm.t_empty[s], kEpiWarps);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(sm.tmem_base)),
+                 "r"(256));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sm.tmem_base;
+
+  if (warp == kEpiWarps) {
+    // ---------------- G^T staging (bf16, swizzled, rows = outputs n) and column sums ----------------
+    long long slice = b0 / bps;
+    int bq = (int)(b0 - slice * bps);
+    int gcount = 0;
+    for (int i = 0; i < n_blocks; ++i) {
+      if (i == 0 || bq == 0) {
+        const int gb = gcount & 1;
+        mbar_wait(&sm.g_empty[gb], ((uint32_t)(gcount >> 1) & 1u) ^ 1u, a.status);
+        int l, sk, b, h;
+        slice_coords(slice, a.k, l, sk, b, h);
+        const float* Gp = a.G + gauge_set(l, sk, h, a.k) * D * D;  // G[k][n]
+        unsigned char* gdst = sm.gs + gb * kBlockBytes;
+        // lane owns output columns n = lane, lane+32, ...: row n of B = column n of G
+        for (int n = lane; n < D; n += 32) {
+          float cs = 0.0f;
+          for (int k0 = 0; k0 < D; k0 += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float g0 = __ldg(Gp + (k0 + 2 * e) * D + n), g1 = __ldg(Gp + (k0 + 2 * e + 1) * D + n);
+              w[e] = pack_bf16x2(g0, g1);
+              cs += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xffff0000u);
+            }
+            *reinterpret_cast<uint4*>(gdst + sw128_offset(n, k0)) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          sm.colsum[gb * 128 + n] = cs;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.g_full[gb]);
+        ++gcount;
+      }
+      if (++bq == bps) {
+        bq = 0;
+        ++slice;
+      }
+    }
+  } else if (warp == kEpiWarps + 1) {
+    // ---------------- MMA issue ----------------
+    if (lane == 0) {
+      long long slice = b0 / bps;
+      int bq = (int)(b0 - slice * bps);
+      int gcount = 0;
+      for (int i = 0; i < n_blocks; ++i) {
+        const int gb = gcount & 1, ab = i & 1;
+        if (i == 0 || bq == 0) mbar_wait(&sm.g_full[gb], (uint32_t)(gcount >> 1) & 1u, a.status);
+        mbar_wait(&sm.a_full[ab], (uint32_t)(i >> 1) & 1u, a.status);
+        mbar_wait(&sm.t_empty[ab], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.status);
+        tc_fence_after();
+        const uint32_t aa = smem_u32(sm.as + ab * kBlockBytes), ga = smem_u32(sm.gs + gb * kBlockBytes);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t koff = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_bf16(tmem + ab * 128, sw128_desc(aa + koff), sw128_desc(ga + koff), k > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.a_empty[ab]);
+        umma_commit(&sm.t_full[ab]);
+        if ((bq + 1 == bps) || (i + 1 == n_blocks)) {
+          umma_commit(&sm.g_empty[gb]);
+          ++gcount;
+        }
+        if (++bq == bps) {
+          bq = 0;
+          ++slice;
+        }
+      }
+    }
+  } else {
+    // ---------------- code expansion (block i+1) and epilogue (block i); thread = token row ----------------
+    const int row = 32 * warp + lane;
+    long long slice_c = b0 / bps;  // cursor of the block being expanded
+    int bq_c = (int)(b0 - slice_c * bps);
+    long long slice_e = slice_c;   // cursor of the block in the epilogue
+    int bq_e = bq_c;
+    int gcount_e = 0;
+    auto expand = [&](int i) {
+      const int ab = i & 1;
+      mbar_wait(&sm.a_empty[ab], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.status);
+      const int valid = min(128, a.nt - 128 * bq_c);
+      const int tok = a.t0 + 128 * bq_c + min(row, valid - 1);  // rows past the range repeat a valid row
+      const uint4* src = reinterpret_cast<const uint4*>(a.codes_in + slice_c * slice_code_bytes +
+                                                        (long long)(tok / 16) * (16 * D * BITS / 8) +
+                                                        (tok % 16) * (D * BITS / 8));
+      uint32_t words[4 * BITS + 1];
+#pragma unroll
+      for (int w = 0; w < BITS; ++w) {
+        const uint4 v = src[w];
+        words[4 * w] = v.x; words[4 * w + 1] = v.y; words[4 * w + 2] = v.z; words[4 * w + 3] = v.w;
+      }
+      words[4 * BITS] = 0;
+      unsigned char* adst = sm.as + ab * kBlockBytes;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {  // 16-byte chunk c = channels 8c .. 8c+7
+        uint32_t q[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int bit = (8 * c + e) * BITS;
+          q[e] = __funnelshift_r(words[bit >> 5], words[(bit >> 5) + 1], bit & 31) & M;
+        }
+        const uint4 w = make_uint4(code_pair_bf16(q[0], q[1]), code_pair_bf16(q[2], q[3]), code_pair_bf16(q[4], q[5]),
+                                   code_pair_bf16(q[6], q[7]));
+        *reinterpret_cast<uint4*>(adst + sw128_offset(row, 8 * c)) = w;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.a_full[ab]);
+      if (++bq_c == bps) {
+        bq_c = 0;
+        ++slice_c;
+      }
+    };
+    if (n_blocks > 0) expand(0);
+    for (int i = 0; i < n_blocks; ++i) {
+      if (i + 1 < n_blocks) expand(i + 1);
+      const int ab = i & 1;
+      const int gb = gcount_e & 1;
+      const int valid = min(128, a.nt - 128 * bq_e);
+      const int tok = a.t0 + 128 * bq_e + row;
+      float sf = 0.0f, zf = 0.0f;
+      if (row < valid) {
+        const long long bidx = slice_e * (a.k.T / 16) + tok / 16;
+        sf = __half2float(__ushort_as_half(__ldg(a.scales_in + bidx)));
+        zf = __half2float(__ushort_as_half(__ldg(a.zeros_in + bidx)));
+      }
+      mbar_wait(&sm.t_full[ab], (uint32_t)(i >> 1) & 1u, a.status);
+      tc_fence_after();
+      const uint32_t taddr = tmem + ab * 128 + ((uint32_t)(32 * warp) << 16);
+      const float* cs = sm.colsum + gb * 128;
+      uint4* dst = reinterpret_cast<uint4*>(a.kv_out + (slice_e * a.k.T + tok) * (long long)D);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float v[32];
+        tmem_ld32(taddr + 32 * c4, v);
+        tmem_wait_ld();
+        if (row < valid) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            uint4 o;
+            o.x = pack_bf16x2(__fmaf_rn(sf, v[j + 0], zf * cs[32 * c4 + j + 0]), __fmaf_rn(sf, v[j + 1], zf * cs[32 * c4 + j + 1]));
+            o.y = pack_bf16x2(__fmaf_rn(sf, v[j + 2], zf * cs[32 * c4 + j + 2]), __fmaf_rn(sf, v[j + 3], zf * cs[32 * c4 + j + 3]));
+            o.z = pack_bf16x2(__fmaf_rn(sf, v[j + 4], zf * cs[32 * c4 + j + 4]), __fmaf_rn(sf, v[j + 5], zf * cs[32 * c4 + j + 5]));
+            o.w = pack_bf16x2(__fmaf_rn(sf, v[j + 6], zf * cs[32 * c4 + j + 6]), __fmaf_rn(sf, v[j + 7], zf * cs[32 * c4 + j + 7]));
+            dst[(32 * c4 + j) / 8] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.t_empty[ab]);
+      const bool last_of_slice = (bq_e + 1 == bps) || (i + 1 == n_blocks);
+      if (last_of_slice) {
+        if (lane == 0) mbar_arrive(&sm.g_empty[gb]);
+        ++gcount_e;
+      }
+      if (++bq_e == bps) {
+        bq_e = 0;
+        ++slice_e;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+  }
+}
+
+namespace {
+template <int BITS>
+cudaError_t fh_dec_launch(const CodecArgs& a, int num_sms, cudaStream_t st) {
+  auto kern = fullhead_decode_kernel<BITS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFdSmem);
+  if (e != cudaSuccess) return e;
+  const long long total = (long long)((a.nt + 127) / 128) * a.k.slices();
+  const int grid = (int)(total < num_sms ? total : num_sms);
+  kern<<<grid, kDecThreads, kFdSmem, st>>>(a);
+  return cudaGetLastError();
+}
+}  // namespace
+
+namespace {
+template <int BITS>
+cudaError_t fh_enc_launch(const CodecArgs& a, int num_sms, cudaStream_t st) {
+  alignas(64) CUtensorMap tmap;
+  const uint64_t rows = (uint64_t)a.k.slices() * a.k.T;
+  if (!make_tmap_2d_bf16(&tmap, a.kv, rows, 128, 64, 128)) return cudaErrorInvalidValue;
+  auto kern = fullhead_encode_kernel<BITS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFhSmem);
+  if (e != cudaSuccess) return e;
+  const long long total = (long long)((a.nt + 127) / 128) * a.k.slices();
+  const int grid = (int)(total < num_sms ? total : num_sms);
+  kern<<<grid, kThreads, kFhSmem, st>>>(tmap, a);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_fullhead(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st) {
+  if (a.nt == 0) return cudaSuccess;
+  if (a.k.d != 128 || a.W != 128) return cudaErrorInvalidValue;
+  switch (a.bits) {
+    case 2: return encode ? fh_enc_launch<2>(a, num_sms, st) : fh_dec_launch<2>(a, num_sms, st);
+    case 3: return encode ? fh_enc_launch<3>(a, num_sms, st) : fh_dec_launch<3>(a, num_sms, st);
+    case 4: return encode ? fh_enc_launch<4>(a, num_sms, st) : fh_dec_launch<4>(a, num_sms, st);
+    case 6: return encode ? fh_enc_launch<6>(a, num_sms, st) : fh_dec_launch<6>(a, num_sms, st);
+    case 8: return encode ? fh_enc_launch<8>(a, num_sms, st) : fh_dec_launch<8>(a, num_sms, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace cg

@@ -83,3 +83,42 @@ def kivi_np(codes, scales, zeros, shape, bits):
     vals = dict(codes=c[:, 1].reshape(L, B, H, T, d // 32, 4 * bits), s=s[:, 1].reshape(L, B, H, T, d // 32),
                 z=z[:, 1].reshape(L, B, H, T, d // 32))
     return keys, vals
+
+
+def check_block_codes_valid(c, s_bits, z_bits, y_ref, eps, bits, w):
+    """Codes from a tensor-core gauge: y is only defined to +-eps (fp32 accumulation
+    order is the hardware's), so each decision must be the oracle's exact one
+    wherever the oracle's value is more than eps from a rounding boundary, and a
+    valid rounding of some y' in [y - eps, y + eps] everywhere else.
+
+    c      : [..., nblk, bytes] packed codes, s_bits / z_bits : [..., nblk] fp16 bits
+    y_ref  : [..., T, d] exact gauged values (fp64), eps : [..., T, d] bound
+    Returns (n_values, n_values whose decision was not unique).
+    """
+    from oracle import quant as oq
+    from oracle.fpround import fl16, fl32, F16_MAX
+    qmax = 2 ** bits - 1
+    yb = oq.block_uniform_view(np.asarray(y_ref, np.float64), 16, w)
+    eb = oq.block_uniform_view(np.asarray(eps, np.float64), 16, w)
+    q = oq.unpack_codes(c, bits, 16 * w)
+    zg = np.asarray(z_bits, np.uint16).view(np.float16).astype(np.float64)
+    sg = np.asarray(s_bits, np.uint16).view(np.float16).astype(np.float64)
+    em = eb.max(axis=-1)
+    mn, mx = yb.min(axis=-1), yb.max(axis=-1)
+    zlo = fl16(np.clip(fl32(mn - em), -F16_MAX, F16_MAX))
+    zhi = fl16(np.clip(fl32(mn + em), -F16_MAX, F16_MAX))
+    assert np.all((zg >= zlo) & (zg <= zhi)), "zero point outside its admissible interval"
+    slo = fl16(np.minimum(fl32(fl32(np.maximum(mx - mn - 2 * em, 0)) / qmax), F16_MAX))
+    shi = fl16(np.minimum(fl32(fl32(mx - mn + 2 * em) / qmax), F16_MAX))
+    assert np.all((sg >= slo) & (sg <= shi)), "step outside its admissible interval"
+    q_lo = oq.quantize(fl32(yb - eb), zg[..., None], sg[..., None], bits)
+    q_hi = oq.quantize(fl32(yb + eb), zg[..., None], sg[..., None], bits)
+    assert np.all((q >= q_lo) & (q <= q_hi)), "code outside its admissible interval"
+    # given the device's (validated) z and s, a code is decided uniquely when its interval is one value
+    unique = q_lo == q_hi
+    q_ref = oq.quantize(fl32(yb), zg[..., None], sg[..., None], bits)
+    assert np.array_equal(q[unique], q_ref[unique])
+    # z and s themselves must be the oracle's wherever their intervals are single values
+    z_ref, s_ref = oq.quant_params(mn, mx, bits)
+    assert np.array_equal(zg[zlo == zhi], z_ref[zlo == zhi]) and np.array_equal(sg[slo == shi], s_ref[slo == shi])
+    return q.size, int((~unique).sum())
