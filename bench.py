@@ -165,6 +165,8 @@ def run_cg(args):
     enc_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
     dec_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
 
+    rows = {} if args.no_rows else measure_rows(args, cg, synth, torch, kv, G, stream, dev, rank)
+
     # --- end to end through the C ABI with host buffers -------------------------------------
     kv_host = kv.cpu().pin_memory()
     out_host = torch.empty(kv.shape, dtype=kv.dtype, pin_memory=True)
@@ -242,11 +244,80 @@ def run_cg(args):
         "e2e": None if args.no_e2e else {"value": round(ws * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                                          "h2d_bytes_per_step": kv_bytes, "d2h_bytes_per_step": kv_bytes},
         "gpu_launches": 2 * args.steps,
+        "rows": rows,
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.bits, budget_s=args.cpu_seconds)
     return line
+
+
+def _time(fn, stream, reps=5, warm=2):
+    import torch
+    for _ in range(warm):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_rows(args, cg, synth, torch, kv, G16, stream, dev, rank):
+    """Per-row kernel timings on the 8B-shaped cache (every other hot-path row), each
+    as ms per call, GB/s of algorithmic traffic and the fraction of the HBM peak."""
+    hbm, _ = _peaks()
+    Lc = kv.shape[0]
+    n = kv.numel()
+    kvd = cg.kv_desc_of(kv)
+    out = torch.empty_like(kv)
+    rows = {}
+
+    def rec(name, ms, bytes_per_value, flops_per_value=None):
+        gbs = bytes_per_value * n / (ms * 1e-3) / 1e9
+        rows[name] = {"ms": round(ms, 4), "alg_GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                      "kv_GBps": round(2 * n / (ms * 1e-3) / 1e9, 1)}
+        if flops_per_value:
+            rows[name]["TFLOPs"] = round(flops_per_value * n / (ms * 1e-3) / 1e12, 1)
+
+    with torch.cuda.stream(stream):
+        for bits in (3, 6):
+            codec = cg.codec_desc(g=16, bits=bits)
+            c, sc, z = cg.alloc_encoded(kvd, codec, device=dev)
+            bpv = 2 + bits / 8 + 4 / 256
+            rec("encode_g16_b%d" % bits, _time(lambda: cg.cg_encode(kvd, codec, kv, G16, 0, T, c, sc, z, None, stream=stream), stream), bpv)
+            rec("decode_g16_b%d" % bits, _time(lambda: cg.cg_decode(kvd, codec, c, sc, z, G16, 0, T, out, stream=stream), stream), bpv)
+        # full-head gauge, G = exp(A - A^T), A ~ N(0, 0.05^2)
+        A = synth.gauge_params(Lc, H, 1, 128, sigma=0.05, seed=rank + 5).to(dev)
+        G128 = torch.empty_like(A)
+        cg.cg_gauge_build(A, G128, stream=stream)
+        codec = cg.codec_desc(g=128, bits=4, range_cols=128)
+        c, sc, z = cg.alloc_encoded(kvd, codec, device=dev)
+        bpv = 2 + 4 / 8 + 4 / (16 * 128)
+        rec("fullhead_encode_b4", _time(lambda: cg.cg_encode(kvd, codec, kv, G128, 0, T, c, sc, z, None, stream=stream), stream), bpv, 256)
+        rec("fullhead_decode_b4", _time(lambda: cg.cg_decode(kvd, codec, c, sc, z, G128, 0, T, out, stream=stream), stream), bpv, 256)
+        # KIVI-style, 3 bits, g = 16 fused
+        codec = cg.codec_desc(g=16, bits=3, mode=cg.KIVI)
+        c, sc, z = cg.alloc_encoded(kvd, codec, device=dev)
+        bpv = 2 + 3 / 8 + 4 / 32
+        rec("kivi_encode_b3", _time(lambda: cg.cg_encode(kvd, codec, kv, G16, 0, T, c, sc, z, None, stream=stream), stream), bpv)
+        rec("kivi_decode_b3", _time(lambda: cg.cg_decode(kvd, codec, c, sc, z, G16, 0, T, out, stream=stream), stream), bpv)
+        # append: one 128-token chunk of every head (a decode step of the rolling cache)
+        rec("kivi_append_128tok", _time(lambda: cg.cg_encode(kvd, codec, kv, G16, T - 128, 128, c, sc, z, None, stream=stream), stream, reps=20), bpv * 128 / T)
+        # spectral statistics of one 4096-token window: forward, and forward + dL/dG
+        st = cg.StatsDesc(16, 16, 0, 1.0, 0.02, 0.04)
+        nblk = n // (16 * 128)
+        lf = torch.empty(nblk, dtype=torch.float32, device=dev)
+        lr = torch.empty_like(lf)
+        tot = torch.empty(4, dtype=torch.float64, device=dev)
+        dG = torch.empty_like(G16)
+        ws = torch.empty(max(cg.cg_spectral_workspace_size(kvd, st, True), 16), dtype=torch.uint8, device=dev)
+        rec("stats_fwd", _time(lambda: cg.cg_spectral_stats(kvd, st, kv, G16, lf, lr, tot, None, ws, stream=stream), stream), 2.0, 2 * 144 + 32)
+        rec("stats_fwd_bwd", _time(lambda: cg.cg_spectral_stats(kvd, st, kv, G16, lf, lr, tot, dG, ws, stream=stream), stream), 4.0, 2 * 288 + 96)
+    cg.cg_sync_status(stream)
+    return rows
 
 
 def _traffic_record(kernel, bits):
@@ -345,6 +416,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=L, help="fewer layers for a small profiling case")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row kernel timings")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "cg":
         args.warmup = 3

@@ -180,23 +180,42 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec, const uint
   return from_cuda(launch_group_codec(a, false, num_sms(), (cudaStream_t)stream));
 }
 
-cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* st, int32_t want_grad, uint64_t* bytes) {
-  (void)want_grad;
+static cg_status check_stats(const cg_kv_desc* kv, const cg_stats_desc* st) {
   cg_status s = check_kv(kv);
   if (s != CG_OK) return s;
-  if (!st || !bytes) return CG_ERR_INVALID;
-  return CG_ERR_UNSUPPORTED;
+  if (!st) return CG_ERR_INVALID;
+  if (st->tb != 16) return CG_ERR_UNSUPPORTED;
+  if (kv->d_head != 128 || kv->tokens % 128 != 0) return CG_ERR_UNSUPPORTED;
+  if (st->g != 0 && st->g != 16) return CG_ERR_UNSUPPORTED;
+  if (!(st->tau > 0.0f)) return CG_ERR_INVALID;
+  return CG_OK;
+}
+
+cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* st, int32_t want_grad, uint64_t* bytes) {
+  cg_status s = check_stats(kv, st);
+  if (s != CG_OK) return s;
+  if (!bytes) return CG_ERR_INVALID;
+  *bytes = spectral_workspace_bytes(geom(kv), want_grad != 0);
+  return CG_OK;
 }
 
 cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st, const void* x_dev, const float* G_dev,
                             float* lfreq_dev, float* lrate_dev, double* totals_dev, float* dG_dev, void* workspace_dev,
                             uint64_t workspace_bytes, void* stream) {
-  (void)x_dev; (void)G_dev; (void)lfreq_dev; (void)lrate_dev; (void)totals_dev; (void)dG_dev;
-  (void)workspace_dev; (void)workspace_bytes; (void)stream;
-  cg_status s = check_kv(kv);
+  cg_status s = check_stats(kv, st);
   if (s != CG_OK) return s;
-  if (!st) return CG_ERR_INVALID;
-  return CG_ERR_UNSUPPORTED;
+  if (!x_dev || !lfreq_dev || !lrate_dev || !totals_dev) return CG_ERR_INVALID;
+  if ((G_dev == nullptr) != (st->g == 0)) return CG_ERR_INVALID;
+  if (dG_dev && !G_dev) return CG_ERR_INVALID;
+  if (!aligned16(x_dev) || !aligned16(lfreq_dev) || !aligned16(lrate_dev) || !aligned16(totals_dev) ||
+      (G_dev && !aligned16(G_dev)) || (dG_dev && !aligned16(dG_dev)))
+    return CG_ERR_INVALID;
+  const uint64_t need = spectral_workspace_bytes(geom(kv), dG_dev != nullptr);
+  if (workspace_bytes < need || (need && (!workspace_dev || !aligned16(workspace_dev)))) return CG_ERR_INVALID;
+  unsigned int* status = status_word();
+  if (!status) return CG_ERR_CUDA;
+  return from_cuda(launch_spectral(geom(kv), st->x_is_fp32, x_dev, G_dev, st->lambda_f, st->lambda_r, st->tau, lfreq_dev,
+                                   lrate_dev, totals_dev, dG_dev, workspace_dev, status, num_sms(), (cudaStream_t)stream));
 }
 
 cg_status cg_sync_status(void* stream) {
