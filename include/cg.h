@@ -49,7 +49,8 @@ typedef enum {
   CG_ERR_INVALID = 1,     /* bad argument: null, misaligned, out of range   */
   CG_ERR_UNSUPPORTED = 2, /* valid request this build has no kernel for     */
   CG_ERR_CUDA = 3,        /* launch or runtime error                        */
-  CG_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out             */
+  CG_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out             */
+  CG_ERR_TOO_LARGE = 5    /* request exceeds a fixed, built-in scratch size */
 } cg_status;
 
 typedef enum {
@@ -190,6 +191,34 @@ cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st,
                             float* lfreq_dev, float* lrate_dev, double* totals_dev,
                             float* dG_dev, void* workspace_dev, uint64_t workspace_bytes,
                             void* stream);
+
+/* cg_spectral_stats for callers that cannot allocate device memory.
+ *
+ * No counterpart in the paper: this is a deployment variant of the library.
+ * Some callers are not allowed to allocate: code running inside a host
+ * framework that hands out only pre-planned buffers (serving engines with a
+ * fixed memory plan, plug-ins, real-time loops where cudaMalloc's implicit
+ * synchronization is not acceptable) cannot create the workspace that
+ * cg_spectral_stats needs for its dL/dG partials.  This entry point takes the
+ * same arguments minus the workspace and uses a scratch array compiled into
+ * the library instead (4 MiB per GPU, reserved on every GPU that loads the
+ * library until the process exits).  It allocates nothing.
+ *   Limit: L * 2 * B * H (head slices) <= 512 when dG_dev is given (one 8 KiB
+ *   dG partial per slice, d_head = 128, g = 16); larger requests return
+ *   CG_ERR_TOO_LARGE before anything is enqueued.  Without dG_dev no scratch is
+ *   used and there is no limit.
+ *   Set-up: the first call on a device looks up the scratch array's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture.
+ *   Sharing: all calls on a device share the one scratch array.  Each call
+ *   writes every scratch byte it later reads, so nothing needs clearing, but
+ *   calls whose work overlaps on the GPU (different streams, no ordering) race
+ *   on it and must be serialized by the caller.
+ * Results, layouts and errors are otherwise those of cg_spectral_stats. */
+cg_status cg_spectral_stats_noalloc(const cg_kv_desc* kv, const cg_stats_desc* st,
+                                    const void* x_dev, const float* G_dev,
+                                    float* lfreq_dev, float* lrate_dev, double* totals_dev,
+                                    float* dG_dev, void* stream);
 
 /* Synchronizes `stream`, then reports (and clears) the device status word:
  * CG_ERR_TIMEOUT if a bounded wait ran out since the last check, CG_ERR_CUDA on

@@ -14,12 +14,13 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcg.so")
 
-CG_OK, CG_ERR_INVALID, CG_ERR_UNSUPPORTED, CG_ERR_CUDA, CG_ERR_TIMEOUT = range(5)
+CG_OK, CG_ERR_INVALID, CG_ERR_UNSUPPORTED, CG_ERR_CUDA, CG_ERR_TIMEOUT, CG_ERR_TOO_LARGE = range(6)
 BLOCK_UNIFORM, KIVI = 0, 1
 
 # Every symbol include/cg.h declares.
 EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
-           "cg_spectral_stats", "cg_sync_status", "cg_last_cuda_error", "cg_status_string", "cg_version")
+           "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_sync_status", "cg_last_cuda_error",
+           "cg_status_string", "cg_version")
 
 
 class KvDesc(ctypes.Structure):
@@ -71,13 +72,15 @@ def lib():
                                                  ctypes.POINTER(u64)]
         L.cg_spectral_stats.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(StatsDesc), vp, vp, vp, vp, vp, vp,
                                         vp, u64, vp]
+        L.cg_spectral_stats_noalloc.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(StatsDesc), vp, vp, vp, vp, vp,
+                                                vp, vp]
         L.cg_sync_status.argtypes = [vp]
         L.cg_status_string.argtypes = [ctypes.c_int]
         L.cg_status_string.restype = ctypes.c_char_p
         L.cg_version.restype = ctypes.c_int32
         L.cg_last_cuda_error.restype = ctypes.c_char_p
         for name in ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
-                     "cg_spectral_stats", "cg_sync_status"):
+                     "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_sync_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -189,6 +192,16 @@ def cg_spectral_stats(kvd, st, x, G, lfreq, lrate, totals, dG=None, workspace=No
                                    _ptr(totals, torch.float64, "totals", 4), _ptr(dG, torch.float32, "dG"),
                                    None if workspace is None else ctypes.c_void_p(workspace.data_ptr()),
                                    ws_bytes, _stream(stream)), "cg_spectral_stats")
+
+
+def cg_spectral_stats_noalloc(kvd, st, x, G, lfreq, lrate, totals, dG=None, stream=None):
+    """cg_spectral_stats without a workspace argument: for callers that cannot
+    allocate device memory, the library's built-in scratch array is used."""
+    xdt = torch.float32 if st.x_is_fp32 else torch.bfloat16
+    _check(lib().cg_spectral_stats_noalloc(ctypes.byref(kvd), ctypes.byref(st), _ptr(x, xdt, "x"),
+                                           _ptr(G, torch.float32, "G"), _ptr(lfreq, torch.float32, "lfreq"),
+                                           _ptr(lrate, torch.float32, "lrate"), _ptr(totals, torch.float64, "totals", 4),
+                                           _ptr(dG, torch.float32, "dG"), _stream(stream)), "cg_spectral_stats_noalloc")
 
 
 def cg_sync_status(stream=None):

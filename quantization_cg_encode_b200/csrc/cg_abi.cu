@@ -84,6 +84,23 @@ unsigned int* status_word() {
 
 }  // namespace
 
+namespace cg {
+// Device address of the status word (for entry points defined in other files).
+unsigned int* device_status_word() { return status_word(); }
+
+// Descriptor checks shared by the spectral-statistics entry points.
+cg_status validate_stats(const cg_kv_desc* kv, const cg_stats_desc* st) {
+  cg_status s = check_kv(kv);
+  if (s != CG_OK) return s;
+  if (!st) return CG_ERR_INVALID;
+  if (st->tb != 16) return CG_ERR_UNSUPPORTED;
+  if (kv->d_head != 128 || kv->tokens % 128 != 0) return CG_ERR_UNSUPPORTED;
+  if (st->g != 0 && st->g != 16) return CG_ERR_UNSUPPORTED;
+  if (!(st->tau > 0.0f)) return CG_ERR_INVALID;
+  return CG_OK;
+}
+}  // namespace cg
+
 extern "C" {
 
 cg_status cg_sizes_for(const cg_kv_desc* kv, const cg_codec_desc* codec, cg_sizes* out) {
@@ -180,19 +197,9 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec, const uint
   return from_cuda(launch_group_codec(a, false, num_sms(), (cudaStream_t)stream));
 }
 
-static cg_status check_stats(const cg_kv_desc* kv, const cg_stats_desc* st) {
-  cg_status s = check_kv(kv);
-  if (s != CG_OK) return s;
-  if (!st) return CG_ERR_INVALID;
-  if (st->tb != 16) return CG_ERR_UNSUPPORTED;
-  if (kv->d_head != 128 || kv->tokens % 128 != 0) return CG_ERR_UNSUPPORTED;
-  if (st->g != 0 && st->g != 16) return CG_ERR_UNSUPPORTED;
-  if (!(st->tau > 0.0f)) return CG_ERR_INVALID;
-  return CG_OK;
-}
 
 cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* st, int32_t want_grad, uint64_t* bytes) {
-  cg_status s = check_stats(kv, st);
+  cg_status s = cg::validate_stats(kv, st);
   if (s != CG_OK) return s;
   if (!bytes) return CG_ERR_INVALID;
   *bytes = spectral_workspace_bytes(geom(kv), want_grad != 0);
@@ -202,7 +209,7 @@ cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* 
 cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st, const void* x_dev, const float* G_dev,
                             float* lfreq_dev, float* lrate_dev, double* totals_dev, float* dG_dev, void* workspace_dev,
                             uint64_t workspace_bytes, void* stream) {
-  cg_status s = check_stats(kv, st);
+  cg_status s = cg::validate_stats(kv, st);
   if (s != CG_OK) return s;
   if (!x_dev || !lfreq_dev || !lrate_dev || !totals_dev) return CG_ERR_INVALID;
   if ((G_dev == nullptr) != (st->g == 0)) return CG_ERR_INVALID;
@@ -244,6 +251,7 @@ const char* cg_status_string(cg_status s) {
     case CG_ERR_UNSUPPORTED: return "unsupported configuration";
     case CG_ERR_CUDA: return "CUDA error";
     case CG_ERR_TIMEOUT: return "device wait timed out";
+    case CG_ERR_TOO_LARGE: return "request exceeds the built-in scratch size";
   }
   return "unknown status";
 }

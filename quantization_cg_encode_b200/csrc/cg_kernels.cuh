@@ -29,6 +29,8 @@ cudaError_t launch_decode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_kivi(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
 cudaError_t launch_fullhead(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
 uint64_t spectral_workspace_bytes(const KvGeom& k, bool want_grad);
+unsigned int* device_status_word();
+cg_status validate_stats(const cg_kv_desc* kv, const cg_stats_desc* st);
 cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f, float lambda_r,
                             float tau, float* lfreq, float* lrate, double* totals, float* dG, void* workspace,
                             unsigned int* status, int num_sms, cudaStream_t st);
