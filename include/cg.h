@@ -58,6 +58,14 @@ typedef enum {
   CG_QUANT_KIVI = 1           /* keys per channel, values per token           */
 } cg_quant_mode;
 
+/* Where the gauge contraction of cg_encode runs.  Codes, steps and zero points
+ * do not depend on it; only the optional gauged output does. */
+typedef enum {
+  CG_ENGINE_AUTO = 0,      /* tensor cores where a kernel exists (g = 16 with
+                              d = 128 and W = g, and g = d), else CUDA cores */
+  CG_ENGINE_CUDA_CORES = 1 /* the fp32 FMA chain on CUDA cores (g < d only)  */
+} cg_engine;
+
 /* Shape of a KV cache: K_l, V_l in R^{B x H x T x d} for l = 1..L
  * (Codec-Gauge, Problem statement and overview).  `tokens` is the capacity T
  * of the buffer; encode/decode take a token range inside it. */
@@ -78,6 +86,7 @@ typedef struct {
  *               (the page's "one range per T_b x d_l block").
  *   mode        cg_quant_mode.
  *   kivi_key_tokens, kivi_val_channels: KIVI group sizes, both 32.
+ *   engine      cg_engine (encode only).
  */
 typedef struct {
   int32_t g;
@@ -87,6 +96,7 @@ typedef struct {
   int32_t mode;
   int32_t kivi_key_tokens;
   int32_t kivi_val_channels;
+  int32_t engine;
 } cg_codec_desc;
 
 /* Buffer sizes of an encoded cache (whole capacity T).  The zero-point and
@@ -149,7 +159,15 @@ cg_status cg_gauge_build(const float* A_dev, float* G_dev, int32_t n_mats, int32
  * q = clamp(rne(fl32(fl32(y - z) * fl32(1/s))), 0, 2^b - 1), q = 0 if s = 0.
  * Gauged values: for g < d each y_i is the fp32 fused-multiply-add chain over
  * j = 0..g-1 in index order (bit-reproducible); for g = d the contraction runs
- * on the tensor cores with G rounded to bf16 and fp32 accumulation. */
+ * on the tensor cores with G rounded to bf16 and fp32 accumulation.
+ * For g < d the codes, steps and zero points are those of the chain whatever
+ * the engine: the tensor-core encoder (g = 16, d = 128, W = g) contracts with
+ * G split exactly into three bf16 terms and re-evaluates the chain wherever
+ * the tensor-core value could change a decision, which relies on G having
+ * orthonormal rows (checked per head slice; a gauge that is not orthogonal to
+ * 2^-12 is evaluated with the chain throughout).  Its gauged output then
+ * holds the values it quantized: within 2^-16 max|y| of the block (16 x 16)
+ * of the chain, and equal to it wherever the chain was evaluated. */
 cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec,
                     const void* kv_dev, const float* G_dev, int32_t t0, int32_t nt,
                     uint8_t* codes_dev, void* scales_dev, void* zeros_dev,

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libcg.so")
 
 CG_OK, CG_ERR_INVALID, CG_ERR_UNSUPPORTED, CG_ERR_CUDA, CG_ERR_TIMEOUT, CG_ERR_TOO_LARGE = range(6)
 BLOCK_UNIFORM, KIVI = 0, 1
+ENGINE_AUTO, ENGINE_CUDA_CORES = 0, 1
 
 # Every symbol include/cg.h declares.
 EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
@@ -31,7 +32,8 @@ class KvDesc(ctypes.Structure):
 class CodecDesc(ctypes.Structure):
     _fields_ = [("g", ctypes.c_int32), ("bits", ctypes.c_int32), ("tb", ctypes.c_int32),
                 ("range_cols", ctypes.c_int32), ("mode", ctypes.c_int32),
-                ("kivi_key_tokens", ctypes.c_int32), ("kivi_val_channels", ctypes.c_int32)]
+                ("kivi_key_tokens", ctypes.c_int32), ("kivi_val_channels", ctypes.c_int32),
+                ("engine", ctypes.c_int32)]
 
 
 class Sizes(ctypes.Structure):
@@ -119,8 +121,10 @@ def kv_desc(layers, batch, heads, tokens, d_head):
     return KvDesc(layers, batch, heads, tokens, d_head)
 
 
-def codec_desc(g=16, bits=4, tb=16, range_cols=None, mode=BLOCK_UNIFORM, kivi_key_tokens=32, kivi_val_channels=32):
-    return CodecDesc(g, bits, tb, g if range_cols is None else range_cols, mode, kivi_key_tokens, kivi_val_channels)
+def codec_desc(g=16, bits=4, tb=16, range_cols=None, mode=BLOCK_UNIFORM, kivi_key_tokens=32, kivi_val_channels=32,
+               engine=ENGINE_AUTO):
+    return CodecDesc(g, bits, tb, g if range_cols is None else range_cols, mode, kivi_key_tokens, kivi_val_channels,
+                     engine)
 
 
 def kv_desc_of(kv):

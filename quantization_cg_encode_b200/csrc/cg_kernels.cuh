@@ -25,6 +25,8 @@ struct CodecArgs {
 
 cudaError_t launch_group_codec(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
 cudaError_t launch_encode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
+bool encode_tc16_supported(const CodecArgs& a);
+cudaError_t launch_encode_tc16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_decode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_kivi(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
 cudaError_t launch_fullhead(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);

@@ -41,6 +41,12 @@ def run_decode(kv_shape, G, codec, codes, scales, zeros, t0=0, nt=None, fill=0.0
     return out
 
 
+def tensor_core_g16(shape, codec):
+    """True when cg_encode runs the tensor-core g = 16 encoder for this request."""
+    return (codec.g == 16 and shape[-1] == 128 and codec.range_cols == 16 and codec.mode == cg.BLOCK_UNIFORM
+            and codec.engine == cg.ENGINE_AUTO)
+
+
 def block_uniform_np(codes, scales, zeros, shape, codec):
     """Device buffers -> numpy views [L,2,B,H,T/16,d/W,bytes] and [L,2,B,H,T/16,d/W]."""
     L, _, B, H, T, d = shape

@@ -13,7 +13,8 @@ from oracle import codec as oc
 from oracle import gauge as og
 from oracle import quant as oq
 from quantization_cg_encode_b200 import cg, synth
-from tests.gpu_util import (assert_close_bf16, bf16_np, block_uniform_np, need_gpu, run_decode, run_encode)
+from tests.gpu_util import (assert_close_bf16, bf16_np, block_uniform_np, need_gpu, run_decode, run_encode,
+                            tensor_core_g16)
 
 pytestmark = pytest.mark.gpu
 
@@ -39,7 +40,14 @@ def _check_encode(kv, G, codec, t0=0, nt=None):
     c, s, z = block_uniform_np(codes, scales, zeros, kv.shape, codec)
     tb0, tb1 = t0 // 16, (t0 + nt) // 16
     y = gauged.cpu().numpy().astype(np.float64)
-    assert np.array_equal(y[..., t0:t0 + nt, :], ref["y"]), "gauged values differ from the fp32 chain"
+    if tensor_core_g16(kv.shape, codec):
+        # the tensor-core encoder reports the values it quantized: within 2^-16 of the
+        # block maximum from the chain (its codes are the chain's, checked below)
+        d = oq.block_uniform_view(np.abs(y[..., t0:t0 + nt, :] - ref["y"]), 16, 16).max(-1)
+        m = oq.block_uniform_view(np.abs(ref["y"]), 16, 16).max(-1)
+        assert np.all(d <= 2.0 ** -16 * m), "gauged values beyond the tensor-core bound"
+    else:
+        assert np.array_equal(y[..., t0:t0 + nt, :], ref["y"]), "gauged values differ from the fp32 chain"
     assert np.all(np.isnan(y[..., :t0, :])) and np.all(np.isnan(y[..., t0 + nt:, :])), "wrote outside the range"
     assert np.array_equal(z[..., tb0:tb1, :], np.asarray(ref["z"]).astype(np.float16).view(np.uint16))
     assert np.array_equal(s[..., tb0:tb1, :], np.asarray(ref["s"]).astype(np.float16).view(np.uint16))
