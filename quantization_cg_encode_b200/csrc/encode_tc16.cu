@@ -54,8 +54,8 @@
 //     = token row): tcgen05.ld, per-group row ranges, a transposing half-warp
 //     reduction that leaves block (tile, r) on lanes 2r, 2r+1 of the tile's
 //     half-warp, which compute its parameters once; then quantize, check,
-//     pack and store.  The x stage is released after the epilogue (the chain
-//     reads x from it).
+//     pack and store; the chain, where needed, reads x from global memory
+//     (the x stage is released as soon as the tensor cores have read it).
 // Every wait on an mbarrier is bounded in time.
 #include <cuda.h>
 
@@ -132,6 +132,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Mark v as written here, so that no use of v can be scheduled before this
+// point (a TMEM load writes its registers asynchronously, until the wait).
+__device__ __forceinline__ void reg_fence16(float* v) {
+  asm volatile(""
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]));
+}
+// Wait for this thread's TMEM loads; the n floats at v (n = 16 or 32) were
+// their destination.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_into(float* v) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  reg_fence16(v);
+  if constexpr (N == 32) reg_fence16(v + 16);
+}
 
 __device__ __forceinline__ float min3f(float a, float b, float c) {
   float r;
@@ -174,17 +189,13 @@ __device__ __forceinline__ uint16_t s_bits(float rng, double inv_qmax) {
   return __half_as_ushort(__float2half_rn(fminf(s32, 65504.0f)));
 }
 
-// Byte offset of element (row, col) in a 128-row x 128-column bf16 block held
-// as two 64-column halves in the 128-byte swizzled layout the TMA writes.
-__device__ __forceinline__ uint32_t xs_offset(int row, int col) {
-  return (col >> 6) * 16384 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2;
-}
-
-// The exact gauged value: output i of group r for token row `row` of the
-// staged block, as the fp32 FMA chain in index order from +0.
-__device__ __forceinline__ float chain_y(const unsigned char* xs, const float* gf, int row, int r, int i) {
-  const uint4 c0 = *reinterpret_cast<const uint4*>(xs + xs_offset(row, 16 * r));
-  const uint4 c1 = *reinterpret_cast<const uint4*>(xs + xs_offset(row, 16 * r + 8));
+// The exact gauged value: output i of group r of the token whose 128 bf16
+// channels start at xrow, as the fp32 FMA chain in index order from +0.  (x
+// comes from global memory, most likely L2: the shared-memory copy of the
+// block is released as soon as the tensor cores have read it.)
+__device__ __forceinline__ float chain_y(const uint16_t* xrow, const float* gf, int r, int i) {
+  const uint4 c0 = __ldg(reinterpret_cast<const uint4*>(xrow + 16 * r));
+  const uint4 c1 = __ldg(reinterpret_cast<const uint4*>(xrow + 16 * r + 8));
   const float4* g = reinterpret_cast<const float4*>(gf + (16 * r + i) * 16);
   const float4 g0 = g[0], g1 = g[1], g2 = g[2], g3 = g[3];
   float acc = 0.0f;
@@ -289,6 +300,113 @@ __device__ __forceinline__ float quant16(const float (&y)[16], float zf, float i
   return fmx;
 }
 
+// Exact range of the undecided blocks of a warp (bit lane 2r + 16 h of `und`:
+// block (tile h, group r)): every value within 2A of a block's tensor-core
+// minimum (maximum) is re-evaluated with the chain (the exact extreme is among
+// them, since no other value can lie below min_tc + A), then the block range
+// is reduced again.  Returns this lane's (mn, mx), exact where its block was
+// undecided.  Called by the whole warp; out of line, as it is rarely needed.
+__device__ __noinline__ float2 exact_range(const uint16_t* xrow, const float* gf, uint32_t taddr, uint32_t und,
+                                           float mn, float mx, float A) {
+  const unsigned FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31, r_own = (lane & 15) >> 1;
+  uint32_t gm = 0;
+  for (uint32_t m = und; m; m &= m - 1) gm |= 1u << (((__ffs(m) - 1) & 15) >> 1);
+  while (gm) {
+    const int r = __ffs(gm) - 1;
+    gm &= gm - 1;
+    const int src = (lane & 16) + 2 * r;
+    const float bmn = __shfl_sync(FULL, mn, src), bmx = __shfl_sync(FULL, mx, src);
+    const float bA = __shfl_sync(FULL, A, src);
+    const bool bund = (und >> src) & 1u;
+    float y[16];
+    tmem_ld16(taddr + 16 * r, y);
+    tmem_wait_ld();
+    float lo_t = __int_as_float(0xff800000), hi_t = __int_as_float(0x7f800000);
+    if (bund) {
+      lo_t = __fadd_ru(bmn, __fmul_ru(2.0f, bA));
+      hi_t = __fsub_rd(bmx, __fmul_ru(2.0f, bA));
+    }
+    uint32_t cand = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) cand |= (y[k] <= lo_t || y[k] >= hi_t) ? (1u << k) : 0u;
+    while (__any_sync(FULL, cand != 0)) {
+      if (cand) {
+        const int k0 = __ffs(cand) - 1;
+        cand &= cand - 1;
+        const float e = chain_y(xrow, gf, r, k0);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          if (k == k0) y[k] = e;
+      }
+    }
+    float emn, emx;
+    minmax16(y, emn, emx);
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) {
+      emn = fminf(emn, __shfl_xor_sync(FULL, emn, o));
+      emx = fmaxf(emx, __shfl_xor_sync(FULL, emx, o));
+    }
+    if (bund && r_own == r) {
+      mn = emn;
+      mx = emx;
+    }
+  }
+  return make_float2(mn, mx);
+}
+
+// One row of a group on the slow path: quantize with clamping where the block
+// needs it (th < -2 carries that, with the margin shifted by -4), re-evaluate
+// the chain for every value within the margin of a rounding boundary, pack and
+// store.  Reloads the group's accumulator columns.  Called by the whole warp;
+// out of line, as it is rarely needed.
+template <int BITS>
+__device__ __noinline__ void slow_group(const uint16_t* xrow, const float* gf, uint32_t taddr_r, int r, float zf,
+                                        float inv, float th, bool tile_ok, uint8_t* crow_r, float* grow) {
+  constexpr int QMAX = (1 << BITS) - 1;
+  const unsigned FULL = 0xffffffffu;
+  float y[16];
+  tmem_ld16(taddr_r, y);
+  tmem_wait_ld();
+  const bool clamp = th < -2.0f;
+  if (clamp) th += 4.0f;
+  const float nzi = -zf * inv;  // as in quant16
+  uint32_t rb[16];
+  uint32_t pend = 0;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float t = __fmaf_rn(y[k], inv, nzi);
+    if (clamp) t = fminf(fmaxf(t, 0.0f), (float)QMAX);
+    const float rr = __fadd_rn(t, kMagic);
+    rb[k] = __float_as_uint(rr);
+    if (tile_ok && fabsf(__fsub_rn(t, __fsub_rn(rr, kMagic))) >= th) pend |= 1u << k;
+  }
+  while (__any_sync(FULL, pend != 0)) {
+    if (pend) {
+      const int k0 = __ffs(pend) - 1;
+      pend &= pend - 1;
+      const float e = chain_y(xrow, gf, r, k0);
+      float t = __fmul_rn(__fsub_rn(e, zf), inv);
+      t = fminf(fmaxf(t, 0.0f), (float)QMAX);
+      const uint32_t rr = __float_as_uint(__fadd_rn(t, kMagic));
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        if (k == k0) {
+          rb[k] = rr;
+          y[k] = e;
+        }
+    }
+  }
+  if (tile_ok) {
+    store_row16<BITS>(crow_r, rb);
+    if (grow) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        reinterpret_cast<float4*>(grow)[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+    }
+  }
+}
+
 struct TcSmem {
   unsigned char* xs;  // kXStages x 32 KB, 1024-aligned
   unsigned char* bs;  // 2 x 12 KB bf16 terms, 1024-aligned
@@ -350,7 +468,7 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
   if (threadIdx.x == 0) {
     for (int s = 0; s < kXStages; ++s) {
       mbar_init(&sm.x_full[s], 1);
-      mbar_init(&sm.x_empty[s], 4);  // the four warps of the warpgroup that took the block
+      mbar_init(&sm.x_empty[s], 1);  // released when the tensor cores have read the block
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.g_full[s], 1);
@@ -512,6 +630,7 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
             umma_bf16_n16(tmem + buf * 128 + 16 * r, sw128_desc(xa + (r >> 2) * 16384 + (r & 3) * 32),
                           sw128_desc(ba + (2 * k + (r >> 2)) * 2048 + (r & 3) * 32), k == 2 ? 0u : 1u);
         }
+        umma_commit(&sm.x_empty[s]);
         umma_commit(&sm.t_full[buf]);
         const bool last_of_slice = (bq + 1 == bps) || (i + 1 == n_blocks);
         if (last_of_slice) {
@@ -542,29 +661,35 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
       if (i == 0 || bq == 0) mbar_wait(&sm.k_full[gb], (uint32_t)(gcount >> 1) & 1u, a.status);
       const bool last_of_slice = (bq + 1 == bps) || (i + 1 == n_blocks);
       if (i % kEpiGroups == wg) {
-        const int buf = i & 3, s = i % kXStages;
+        const int buf = i & 3;
         mbar_wait(&sm.t_full[buf], (uint32_t)(i >> 2) & 1u, a.status);
-        mbar_wait(&sm.x_full[s], (uint32_t)(i / kXStages) & 1u, a.status);
         tc_fence_after();
-        const unsigned char* xs = sm.xs + s * kXBytes;
         const float* gf = sm.gf + gb * 2048;
         const float kA = sm.ka[gb];
         const int valid = min(128, a.nt - 128 * bq);
         const bool tile_ok = row < valid;  // valid is a multiple of 16: whole half-warps agree
         const int tok = a.t0 + 128 * bq + row;
+        // the token's input channels, for the chain (an address only: valid rows read it)
+        const uint16_t* xrow = a.kv + (slice * a.k.T + (tile_ok ? tok : a.t0)) * D;
         const long long tile = slice * (a.k.T / 16) + tok / 16;
         const uint32_t taddr = tmem + buf * 128 + ((uint32_t)(32 * quarter) << 16);
 
         // ---- pass 1: row ranges of the 8 groups, then the block ranges ----
         float mnr[8], mxr[8], ssr[8];
+        {
+          float va[32], vb[32];  // two groups at a time; the next two load meanwhile
+          tmem_ld32(taddr, va);
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          float v[64];
-          tmem_ld32(taddr + 64 * c2, v);
-          tmem_ld32(taddr + 64 * c2 + 32, v + 32);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 4; ++h) stats16(v + 16 * h, mnr[4 * c2 + h], mxr[4 * c2 + h], ssr[4 * c2 + h]);
+          for (int c = 0; c < 4; c += 2) {
+            tmem_wait_ld_into<32>(va);
+            tmem_ld32(taddr + 32 * (c + 1), vb);
+            stats16(va, mnr[2 * c], mxr[2 * c], ssr[2 * c]);
+            stats16(va + 16, mnr[2 * c + 1], mxr[2 * c + 1], ssr[2 * c + 1]);
+            tmem_wait_ld_into<32>(vb);
+            if (c + 2 < 4) tmem_ld32(taddr + 32 * (c + 2), va);
+            stats16(vb, mnr[2 * c + 2], mxr[2 * c + 2], ssr[2 * c + 2]);
+            stats16(vb + 16, mnr[2 * c + 3], mxr[2 * c + 3], ssr[2 * c + 3]);
+          }
         }
         // transposing reduction over the 16 rows of a tile (min, max, and the
         // largest row norm): after it, lanes 2r and 2r+1 of each half-warp
@@ -617,50 +742,9 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
         }
         const uint32_t und = __ballot_sync(FULL, (lane & 1) == 0 && !decided && tile_ok);
         if (und) {
-          // exact range of the undecided blocks: re-evaluate every value that
-          // can be the block's minimum or maximum, then reduce again
-          uint32_t gm = 0;
-          for (uint32_t m = und; m; m &= m - 1) gm |= 1u << (((__ffs(m) - 1) & 15) >> 1);
-          while (gm) {
-            const int r = __ffs(gm) - 1;
-            gm &= gm - 1;
-            const int src = (lane & 16) + 2 * r;
-            const float bmn = __shfl_sync(FULL, mn, src), bmx = __shfl_sync(FULL, mx, src);
-            const float bA = __shfl_sync(FULL, A, src);
-            const bool bund = (und >> src) & 1u;
-            float y[16];
-            tmem_ld16(taddr + 16 * r, y);
-            tmem_wait_ld();
-            float lo_t = __int_as_float(0xff800000), hi_t = __int_as_float(0x7f800000);
-            if (bund) {
-              lo_t = __fadd_ru(bmn, __fmul_ru(2.0f, bA));
-              hi_t = __fsub_rd(bmx, __fmul_ru(2.0f, bA));
-            }
-            uint32_t cand = 0;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) cand |= (y[k] <= lo_t || y[k] >= hi_t) ? (1u << k) : 0u;
-            while (__any_sync(FULL, cand != 0)) {
-              if (cand) {
-                const int k0 = __ffs(cand) - 1;
-                cand &= cand - 1;
-                const float e = chain_y(xs, gf, row, r, k0);
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                  if (k == k0) y[k] = e;
-              }
-            }
-            float emn, emx;
-            minmax16(y, emn, emx);
-#pragma unroll
-            for (int o = 8; o >= 1; o >>= 1) {
-              emn = fminf(emn, __shfl_xor_sync(FULL, emn, o));
-              emx = fmaxf(emx, __shfl_xor_sync(FULL, emx, o));
-            }
-            if (bund && r_own == r) {
-              mn = emn;
-              mx = emx;
-            }
-          }
+          const float2 e = exact_range(xrow, gf, taddr, und, mn, mx, A);
+          mn = e.x;
+          mx = e.y;
         }
         const QParams qp = quant_params(mn, mx, inv_qmax);
         // decision margin in t units, and whether the block needs clamping
@@ -692,48 +776,20 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
           const int src = (lane & 16) + 2 * r;
           const float zf = __shfl_sync(FULL, qp.zf, src);
           const float inv = __shfl_sync(FULL, qp.inv, src);
-          float th = __shfl_sync(FULL, thr, src);
-          tmem_wait_ld();
-          const bool clamp = th < -2.0f;
-          if (clamp) th += 4.0f;
+          const float th = __shfl_sync(FULL, thr, src);
+          tmem_wait_ld_into<16>(y);
           uint32_t rb[16];
-          const float fmx = clamp ? quant16<true, QMAX>(y, zf, inv, rb) : quant16<false, QMAX>(y, zf, inv, rb);
-          const bool need = tile_ok && fmx >= th;
-          if (__any_sync(FULL, need)) {
-            uint32_t pend = 0;
-            if (need) {
-#pragma unroll
-              const float nzi = -zf * inv;
-              for (int k = 0; k < 16; ++k) {
-                float t = __fmaf_rn(y[k], inv, nzi);  // as in quant16
-                if (clamp) t = fminf(fmaxf(t, 0.0f), (float)QMAX);
-                const float rr = __fadd_rn(t, kMagic);
-                if (fabsf(__fsub_rn(t, __fsub_rn(rr, kMagic))) >= th) pend |= 1u << k;
-              }
-            }
-            while (__any_sync(FULL, pend != 0)) {
-              if (pend) {
-                const int k0 = __ffs(pend) - 1;
-                pend &= pend - 1;
-                const float e = chain_y(xs, gf, row, r, k0);
-                float t = __fmul_rn(__fsub_rn(e, zf), inv);
-                t = fminf(fmaxf(t, 0.0f), (float)QMAX);
-                const uint32_t rr = __float_as_uint(__fadd_rn(t, kMagic));
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                  if (k == k0) {
-                    rb[k] = rr;
-                    y[k] = e;
-                  }
-              }
-            }
-          }
-          if (tile_ok) {
+          const float fmx = quant16<false, QMAX>(y, zf, inv, rb);
+          float* grow = a.gauged ? a.gauged + (slice * a.k.T + tok) * D + 16 * r : nullptr;
+          if (__any_sync(FULL, tile_ok && (th < -2.0f || fmx >= th))) {
+            // a block needs clamping or holds values near a rounding boundary
+            slow_group<BITS>(xrow, gf, taddr + 16 * r, r, zf, inv, th, tile_ok, crow + r * (32 * BITS), grow);
+          } else if (tile_ok) {
             store_row16<BITS>(crow + r * (32 * BITS), rb);
-            if (a.gauged) {
-              float4* gd = reinterpret_cast<float4*>(a.gauged + (slice * a.k.T + tok) * D + 16 * r);
+            if (grow) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k) gd[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+              for (int k = 0; k < 4; ++k)
+                reinterpret_cast<float4*>(grow)[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
             }
           }
         }
@@ -741,7 +797,6 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&sm.t_empty[buf]);
-          mbar_arrive(&sm.x_empty[s]);
         }
       }
       if (last_of_slice) {
