@@ -184,9 +184,17 @@ __device__ __forceinline__ void stats16(const float* y, float& mn, float& mx, fl
 __device__ __forceinline__ uint16_t z_bits(float mn) {
   return __half_as_ushort(__float2half_rn(fminf(fmaxf(mn, -65504.0f), 65504.0f)));
 }
-__device__ __forceinline__ uint16_t s_bits(float rng, double inv_qmax) {
-  const float s32 = __double2float_rn(__dmul_rn((double)rng, inv_qmax));
-  return __half_as_ushort(__float2half_rn(fminf(s32, 65504.0f)));
+// The step from a range width: fp16(min(fl32(rng / qmax), 65504)).  The fp32
+// quotient is q0 = fl(rng c), c = fl(1/qmax), corrected once with the exact
+// residual fma(-q0, qmax, rng): for qmax = 3, 7, 15, 63 and 255 this equals the
+// correctly rounded rng / qmax for every fp32 rng (checked exhaustively over
+// all 2^31 non-negative values, and odd-symmetric).
+template <int QMAX>
+__device__ __forceinline__ uint16_t s_bits(float rng) {
+  constexpr float c = (float)(1.0 / QMAX);
+  const float q0 = __fmul_rn(rng, c);
+  const float q = __fmaf_rn(__fmaf_rn(-q0, (float)QMAX, rng), c, q0);
+  return __half_as_ushort(__float2half_rn(fminf(q, 65504.0f)));
 }
 
 // The exact gauged value: output i of group r of the token whose 128 bf16
@@ -620,15 +628,19 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
         mbar_wait(&sm.x_full[s], (uint32_t)(i / kXStages) & 1u, a.status);
         mbar_wait(&sm.t_empty[buf], ((uint32_t)(i >> 2) & 1u) ^ 1u, a.status);
         tc_fence_after();
-        const uint32_t xa = smem_u32(sm.xs + s * kXBytes), ba = smem_u32(sm.bs + gb * kBBytes);
+        // descriptors of the stage's x block and of the slice's B terms; an
+        // operand at byte offset o is the descriptor plus o / 16 (start-address field)
+        const uint64_t xd = sw128_desc(smem_u32(sm.xs + s * kXBytes));
+        const uint64_t bd = sw128_desc(smem_u32(sm.bs + gb * kBBytes));
+        const uint32_t td = tmem + buf * 128;
         // lo, mid, hi (small terms first); consecutive MMAs write different groups'
         // accumulators, so they do not wait for one another
 #pragma unroll
         for (int k = 2; k >= 0; --k) {
 #pragma unroll
           for (int r = 0; r < 8; ++r)
-            umma_bf16_n16(tmem + buf * 128 + 16 * r, sw128_desc(xa + (r >> 2) * 16384 + (r & 3) * 32),
-                          sw128_desc(ba + (2 * k + (r >> 2)) * 2048 + (r & 3) * 32), k == 2 ? 0u : 1u);
+            umma_bf16_n16(td + 16 * r, xd + (((r >> 2) * 16384 + (r & 3) * 32) >> 4),
+                          bd + (((2 * k + (r >> 2)) * 2048 + (r & 3) * 32) >> 4), k == 2 ? 0u : 1u);
         }
         umma_commit(&sm.x_empty[s]);
         umma_commit(&sm.t_full[buf]);
@@ -651,7 +663,6 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
     const int j16 = lane & 15;
     const int r_own = j16 >> 1;  // group whose block parameters this lane computes
     const unsigned FULL = 0xffffffffu;
-    const double inv_qmax = 1.0 / (double)QMAX;
     const long long slice_code_bytes = (long long)a.k.T * D * BITS / 8;
     long long slice = b0 / bps;
     int bq = (int)(b0 - slice * bps);
@@ -733,12 +744,16 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
         const float M = fmaxf(fabsf(mn), fabsf(mx));
         const bool finite_bound = kA < 1.0f;
         const float A = finite_bound ? __fmul_ru(kA, __fsqrt_ru(ss)) : __int_as_float(0x7f800000);
+        // z and s are decided when both ends of the interval the exact extreme lies in
+        // give the same fp16 values (the maps are monotone)
         bool decided = false;
+        uint16_t zh = 0, sh = 0;
         if (finite_bound) {
           const float lo_mn = __fsub_rd(mn, A), hi_mn = __fadd_ru(mn, A);
           const float lo_mx = __fsub_rd(mx, A), hi_mx = __fadd_ru(mx, A);
-          decided = z_bits(lo_mn) == z_bits(hi_mn) &&
-                    s_bits(__fsub_rd(lo_mx, hi_mn), inv_qmax) == s_bits(__fsub_ru(hi_mx, lo_mn), inv_qmax);
+          zh = z_bits(lo_mn);
+          sh = s_bits<QMAX>(__fsub_rd(lo_mx, hi_mn));
+          decided = zh == z_bits(hi_mn) && sh == s_bits<QMAX>(__fsub_ru(hi_mx, lo_mn));
         }
         const uint32_t und = __ballot_sync(FULL, (lane & 1) == 0 && !decided && tile_ok);
         if (und) {
@@ -746,7 +761,16 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
           mn = e.x;
           mx = e.y;
         }
-        const QParams qp = quant_params(mn, mx, inv_qmax);
+        if (!decided) {  // mn, mx exact now (or the block is not written)
+          zh = z_bits(mn);
+          sh = s_bits<QMAX>(__fsub_rn(mx, mn));
+        }
+        QParams qp;
+        qp.zh = zh;
+        qp.sh = sh;
+        qp.zf = __half2float(__ushort_as_half(zh));
+        qp.sf = __half2float(__ushort_as_half(sh));
+        qp.inv = (qp.sf != 0.0f) ? __frcp_rn(qp.sf) : 0.0f;
         // decision margin in t units, and whether the block needs clamping
         float thr;
         {
