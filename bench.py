@@ -321,12 +321,18 @@ def measure_rows(args, cg, synth, torch, kv, G16, stream, dev, rank):
 
 
 def _traffic_record(kernel, bits):
-    """DRAM bytes per launch from the committed ncu summary, if one matches."""
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+    committed ncu record, or None when there is none for this kernel or its source
+    has changed since the counters were taken."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f)
-        return rec.get("%s_b%d" % (kernel, bits))
+            rec = json.load(f)["%s_b%d" % (kernel, bits)]
+        with open(os.path.join(ROOT, "quantization_cg_encode_b200", "csrc", rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+                return None
+        return int(rec["traffic"])
     except Exception:
         return None
 
