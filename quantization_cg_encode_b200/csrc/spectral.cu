@@ -191,6 +191,16 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
   const uint32_t tmem = *sm.tmem_base;  // columns [0,128): U1 ; [128,256): dX'^T
   const uint32_t id_fwd = idesc_bf16(false, false), id_bwd = idesc_bf16(true, false);
 
+  // normalized radius r_uv of this thread's channel-frequency column (phase C)
+  float rad[16];
+  {
+    const float rv = (float)(tid & 127) / (kD - 1);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const float ru = (float)u / 15.0f;
+      rad[u] = sqrtf(ru * ru + rv * rv) * 0.70710678118654752f;
+    }
+  }
   int it = 0;  // tiles processed by this CTA (mbarrier phases)
   for (long long slice = blockIdx.x; slice < slices; slice += gridDim.x) {
     int l, sk, b, h;
@@ -270,10 +280,16 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
             const int c = 8 * cb + e;
             if (a.has_g) {
               const int r = c >> 4, i = c & 15;
-              const float* gi = sm.Gs + (r * 16 + i) * 16;
+              const float4* gi = reinterpret_cast<const float4*>(sm.Gs + (r * 16 + i) * 16);
               float acc = 0.0f;
 #pragma unroll
-              for (int j = 0; j < 16; ++j) acc = __fmaf_rn(gi[j], x[16 * r + j], acc);
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const float4 g = gi[j4];
+                acc = __fmaf_rn(g.x, x[16 * r + 4 * j4], acc);
+                acc = __fmaf_rn(g.y, x[16 * r + 4 * j4 + 1], acc);
+                acc = __fmaf_rn(g.z, x[16 * r + 4 * j4 + 2], acc);
+                acc = __fmaf_rn(g.w, x[16 * r + 4 * j4 + 3], acc);
+              }
               y8[e] = acc;
             } else {
               y8[e] = x[c];
@@ -311,27 +327,43 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
       named_bar_sync(1, 128);
       {
         const int v = tid;  // channel-frequency column
-        const float rv = (float)v / (kD - 1);
         const int obase = (int)(row0 / 16);  // first block index of this tile
+        const float inv_tau = 1.0f / a.tau;
         for (int kb = 0; kb < kTile / 16; ++kb) {
           float col[16], U[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) col[t] = sm.S[(16 * kb + t) * kSPitch + v];
+          // 16-point DCT-II through its symmetry C[u][15 - t] = (-1)^u C[u][t]:
+          // even u from col[t] + col[15 - t], odd u from col[t] - col[15 - t]
+          float sm8[8], df8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            sm8[t] = col[t] + col[15 - t];
+            df8[t] = col[t] - col[15 - t];
+          }
           float e_sum = 0.0f, f_sum = 0.0f, r_sum = 0.0f;
-          float rad[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
-            float acc = 0.0f;
+            const float4 c0 = reinterpret_cast<const float4*>(sm.C16 + u * 16)[0];
+            const float4 c1 = reinterpret_cast<const float4*>(sm.C16 + u * 16)[1];
+            float h8[8];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) acc = __fmaf_rn(sm.C16[u * 16 + t], col[t], acc);
+            for (int t = 0; t < 8; ++t) h8[t] = (u & 1) ? df8[t] : sm8[t];  // u is a compile-time index
+            float acc = c0.x * h8[0];
+            acc = __fmaf_rn(c0.y, h8[1], acc);
+            acc = __fmaf_rn(c0.z, h8[2], acc);
+            acc = __fmaf_rn(c0.w, h8[3], acc);
+            acc = __fmaf_rn(c1.x, h8[4], acc);
+            acc = __fmaf_rn(c1.y, h8[5], acc);
+            acc = __fmaf_rn(c1.z, h8[6], acc);
+            acc = __fmaf_rn(c1.w, h8[7], acc);
             U[u] = acc;
-            const float ru = (float)u / 15.0f;
-            rad[u] = sqrtf(ru * ru + rv * rv) * 0.70710678118654752f;
             const float e = acc * acc;
             e_sum += e;
             f_sum = __fmaf_rn(rad[u], e, f_sum);
-            r_sum += log1pf(fabsf(acc) / a.tau);
+            r_sum += __log2f(__fmaf_rn(fabsf(acc), inv_tau, 1.0f));  // log1p(|U| / tau) / ln 2
           }
+          r_sum *= 0.69314718055994531f;
           // block reduction over the 128 columns
 #pragma unroll
           for (int o = 16; o >= 1; o >>= 1) {
@@ -363,14 +395,22 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
               const float sg = U[u] > 0.0f ? 1.0f : (U[u] < 0.0f ? -1.0f : 0.0f);
               dU[u] = __fmaf_rn(cf * U[u], rad[u] - lf, cr * sg / (a.tau + fabsf(U[u])));
             }
+            // dU1[t] = sum_u C[u][t] dU[u]: even-u part Ev and odd-u part Od of
+            // t < 8 give dU1[t] = Ev + Od and dU1[15 - t] = Ev - Od
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-              float acc = 0.0f;
+            for (int t = 0; t < 8; ++t) {
+              float ev = 0.0f, od = 0.0f;
 #pragma unroll
-              for (int u = 0; u < 16; ++u) acc = __fmaf_rn(sm.C16[u * 16 + t], dU[u], acc);
-              const uint16_t hi = bf16_rn(acc);
-              *reinterpret_cast<uint16_t*>(sm.ahi + swz(16 * kb + t, v)) = hi;
-              *reinterpret_cast<uint16_t*>(sm.alo + swz(16 * kb + t, v)) = bf16_rn(acc - bf16_f(hi));
+              for (int u = 0; u < 16; u += 2) {
+                ev = __fmaf_rn(sm.C16[u * 16 + t], dU[u], ev);
+                od = __fmaf_rn(sm.C16[(u + 1) * 16 + t], dU[u + 1], od);
+              }
+              const float d0 = ev + od, d1 = ev - od;
+              const uint16_t h0 = bf16_rn(d0), h1 = bf16_rn(d1);
+              *reinterpret_cast<uint16_t*>(sm.ahi + swz(16 * kb + t, v)) = h0;
+              *reinterpret_cast<uint16_t*>(sm.alo + swz(16 * kb + t, v)) = bf16_rn(d0 - bf16_f(h0));
+              *reinterpret_cast<uint16_t*>(sm.ahi + swz(16 * kb + 15 - t, v)) = h1;
+              *reinterpret_cast<uint16_t*>(sm.alo + swz(16 * kb + 15 - t, v)) = bf16_rn(d1 - bf16_f(h1));
             }
           }
           named_bar_sync(1, 128);  // sm.red reused by the next block
@@ -388,7 +428,7 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
         for (int c4 = 0; c4 < 4; ++c4) {
           float v[32];
           ld32(tmem + 128 + 32 * c4 + ((uint32_t)(32 * warp) << 16), v);  // dX'^T row c: tokens 32 c4 ..
-#pragma unroll 4
+#pragma unroll 8
           for (int tt = 0; tt < 32; ++tt) {
             const long long row = row0 + 32 * c4 + tt;
             float xs[16];
