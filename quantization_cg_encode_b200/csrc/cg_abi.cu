@@ -192,6 +192,7 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec, const uint
   a.kv_out = (uint16_t*)kv_out_dev;
   a.status = status_word();
   if (!a.status) return CG_ERR_CUDA;
+  if (a.kivi && kivi_decode_g16_supported(a)) return from_cuda(launch_kivi_decode_g16(a, num_sms(), (cudaStream_t)stream));
   if (a.kivi) return from_cuda(launch_kivi(a, false, num_sms(), (cudaStream_t)stream));
   if (a.g == kv->d_head) {
     if (kv->d_head != 128) return CG_ERR_UNSUPPORTED;

@@ -29,6 +29,8 @@ bool encode_tc16_supported(const CodecArgs& a);
 cudaError_t launch_encode_tc16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_decode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_kivi(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
+bool kivi_decode_g16_supported(const CodecArgs& a);
+cudaError_t launch_kivi_decode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_fullhead(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
 uint64_t spectral_workspace_bytes(const KvGeom& k, bool want_grad);
 unsigned int* device_status_word();

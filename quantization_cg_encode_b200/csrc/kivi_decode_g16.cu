@@ -1,0 +1,298 @@
+// KIVI-style decode for g = 16 and d_head = 128 on the tensor cores: unpack,
+// dequantize and apply G^T per 16-channel group, bf16 out.
+//
+// Codec-Gauge, Experimental setup: KIVI-style backend (keys with one range per
+// channel and 32 tokens, values with one range per token and 32 channels);
+// Method: the inverse gauge restores K and V before attention, explicitly.
+//
+// A warp decodes a unit of 32 tokens x 128 channels of one head slice, whose
+// codes (512 b bytes) and steps / zero points (128 each) are contiguous in
+// both layouts.  Per 16-token tile and group, mma.sync m16n8k16 (fp16 in, fp32
+// accumulate) against G split into fp16 hi + lo (2^-22):
+//   * values: the step and zero point are one per token, so
+//       x_hat_n = s_t sum_c q_c G[c][n] + z_t colsum_n
+//     with the codes themselves as the A operand (integers, exact in fp16);
+//   * keys: the step and zero point vary with the channel, so A is the
+//     dequantized y = s_c q + z_c (fp32), split into fp16 hi + lo, and
+//       x_hat = A_hi G_hi + A_hi G_lo + A_lo G_hi
+//     (a unit whose |y| could leave the fp16 range is scaled by a power of
+//     two, exactly undone afterwards).
+// The k order of A and B is permuted consistently (each thread reads 4
+// adjacent channels).  The bf16 tile goes through a padded shared-memory
+// staging with stmatrix and leaves with full-line 16-byte stores.
+#include "cg_kernels.cuh"
+
+namespace cg {
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kPitch = 2 * 128 + 16;  // staging row: 256 B + 16 B pad (distinct bank groups per 8 rows)
+constexpr int kStg = 32 * kPitch;
+constexpr int kCodeBuf = 512 * 8;     // codes of a unit at up to 8 bits
+// per warp: output staging, then two input buffers (codes + 16 B slack, steps,
+// zero points), then the column sums of G
+constexpr int kInBuf = kCodeBuf + 16 + 2 * 256;
+constexpr int kWarpSmem = kStg + 2 * kInBuf + 512;
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t f16_sub1024(uint32_t biased) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(biased), "r"(0x64006400u));
+  return r;
+}
+// fp16 pair {c_lo, c_hi} of two codes (< 256): 0x6400 | c is exactly 1024 + c
+__device__ __forceinline__ uint32_t f16pair(uint32_t c_lo, uint32_t c_hi) {
+  return f16_sub1024(0x64006400u | c_lo | (c_hi << 16));
+}
+__device__ __forceinline__ uint32_t f16_bits(float x) { return (uint32_t)__half_as_ushort(__float2half_rn(x)); }
+// fp16 hi and lo words of two fp32 values: hi = fp16(v), lo = fp16(v - hi)
+__device__ __forceinline__ void f16_split2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(v0, v1);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(v0 - hf.x, v1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void stmatrix_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
+// 32 bits starting at bit `bit` of the little-endian stream at p (reads two words)
+__device__ __forceinline__ uint32_t bits_at(const unsigned char* p, int bit) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(p) + (bit >> 5);
+  return __funnelshift_r(w[0], w[1], bit & 31);
+}
+
+}  // namespace
+
+template <int BITS>
+__global__ void __launch_bounds__(kWarps * 32, 1) kivi_decode_g16_kernel(CodecArgs a) {
+  constexpr int D = 128, NG = 8;
+  constexpr uint32_t M = (1u << BITS) - 1u;
+  constexpr int UNIT_BYTES = 512 * BITS;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char* base = smem_raw + warp * kWarpSmem;
+  unsigned char* stg = base;
+  float* csum = reinterpret_cast<float*>(base + kStg + 2 * kInBuf);       // 128 column sums of G
+  const uint32_t st_addr =
+      (uint32_t)__cvta_generic_to_shared(stg) + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kPitch + ((lane >> 4) * 8) * 2;
+  const int g4 = lane >> 2, q4 = lane & 3;
+
+  const int ntg = a.nt / 32;
+  const long long units = a.k.slices() * ntg;
+  const long long slice_bytes = (long long)a.k.T * D * BITS / 8;
+  const long long slice_ranges = (long long)a.k.T * D / 32;
+
+  uint32_t bfr[NG][2][2][2];  // [group][n-half][hi/lo][b0/b1], fp16 pairs of G
+  long long loaded = -1;
+  // a unit's codes, steps and zero points (contiguous in both layouts) into input buffer p
+  auto prefetch = [&](long long uu, int p) {
+    const long long sl = uu / ntg;
+    const int tg = a.t0 / 32 + (int)(uu - sl * ntg);
+    unsigned char* ib = base + kStg + p * kInBuf;
+    const unsigned char* src = a.codes_in + sl * slice_bytes + (long long)tg * UNIT_BYTES;
+#pragma unroll
+    for (int k = 0; k < UNIT_BYTES / 512; ++k) cp_async16(ib + 16 * (32 * k + lane), src + 16 * (32 * k + lane));
+    const long long r0 = sl * slice_ranges + (long long)tg * 128;
+    cp_async8(ib + kCodeBuf + 16 + 8 * lane, a.scales_in + r0 + 4 * lane);
+    cp_async8(ib + kCodeBuf + 16 + 256 + 8 * lane, a.zeros_in + r0 + 4 * lane);
+  };
+  const long long ustride = (long long)gridDim.x * kWarps;
+  long long u = (long long)blockIdx.x * kWarps + warp;
+  if (u < units) prefetch(u, 0);
+  cp_async_commit();
+  for (int it = 0; u < units; u += ustride, ++it) {
+    const int p = it & 1;
+    if (u + ustride < units) prefetch(u + ustride, p ^ 1);  // the next unit loads during this one
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    const unsigned char* cbuf = base + kStg + p * kInBuf;
+    const uint16_t* sbuf = reinterpret_cast<const uint16_t*>(cbuf + kCodeBuf + 16);
+    const uint16_t* zbuf = sbuf + 128;
+    const long long slice = u / ntg;
+    const int tgroup = a.t0 / 32 + (int)(u - slice * ntg);
+    int l, sk, b, h;
+    slice_coords(slice, a.k, l, sk, b, h);
+    const bool key = sk == 0;
+    if (slice != loaded) {  // G fragments and column sums of this head slice
+      const float* G0 = a.G + gauge_set(l, sk, h, a.k) * NG * 256;
+#pragma unroll
+      for (int r = 0; r < NG; ++r) {
+        const float* Gr = G0 + r * 256;  // G[c][n], row-major
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+          const int n = 8 * nh + g4;
+          float gv[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) gv[m] = __ldg(Gr + (4 * q4 + m) * 16 + n);
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            hw[m] = f16_bits(gv[m]);
+            lw[m] = f16_bits(gv[m] - __half2float(__ushort_as_half((unsigned short)hw[m])));
+          }
+          bfr[r][nh][0][0] = hw[0] | (hw[1] << 16);
+          bfr[r][nh][0][1] = hw[2] | (hw[3] << 16);
+          bfr[r][nh][1][0] = lw[0] | (lw[1] << 16);
+          bfr[r][nh][1][1] = lw[2] | (lw[3] << 16);
+        }
+      }
+      __syncwarp();
+      for (int e = lane; e < D; e += 32) {
+        const float* Gr = G0 + (e >> 4) * 256 + (e & 15);
+        float acc = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) acc += __ldg(Gr + c * 16);
+        csum[e] = acc;
+      }
+      loaded = slice;
+    }
+    // keys: a power of two that keeps every |y| of the unit inside fp16
+    float kscale = 1.0f, kunscale = 1.0f;
+    if (key) {
+      float big = 0.0f;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int c = 4 * lane + m;
+        const float s = __half2float(__ushort_as_half(sbuf[c])), z = __half2float(__ushort_as_half(zbuf[c]));
+        big = fmaxf(big, fabsf(z) + s * (float)M);
+      }
+      big = warp_max_f32(big);
+      // warp-uniform, exact powers of two; finite fp16 steps and zero points need at most 3 steps
+      for (int it = 0; it < 8 && big * kscale > 16384.0f; ++it) {
+        kscale *= 0.0625f;
+        kunscale *= 16.0f;
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+#pragma unroll
+      for (int r = 0; r < NG; ++r) {
+        uint32_t pk[2][2];  // [n-half][row half], bf16 pairs
+        if (!key) {
+          // values: record (token, 32-channel group r / 2), channels 16 (r & 1) + 4 q4 .. + 3
+          uint32_t afr[4];
+          float sv[2], zv[2];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int t = 16 * tt + g4 + 8 * half;
+            const int bit = ((t * 4 + (r >> 1)) * 32 + 16 * (r & 1) + 4 * q4) * BITS;
+            const uint32_t v = bits_at(cbuf, bit);
+            const uint32_t c0 = v & M, c1 = (v >> BITS) & M, c2 = (v >> (2 * BITS)) & M, c3 = (v >> (3 * BITS)) & M;
+            // k slots 2q, 2q+1 <- channels 4q, 4q+1;  k slots 2q+8, 2q+9 <- channels 4q+2, 4q+3
+            afr[half] = f16pair(c0, c1);
+            afr[2 + half] = f16pair(c2, c3);
+            sv[half] = __half2float(__ushort_as_half(sbuf[t * 4 + (r >> 1)]));
+            zv[half] = __half2float(__ushort_as_half(zbuf[t * 4 + (r >> 1)]));
+          }
+#pragma unroll
+          for (int nh = 0; nh < 2; ++nh) {
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            mma_f16(acc, afr, bfr[r][nh][0][0], bfr[r][nh][0][1]);
+            mma_f16(acc, afr, bfr[r][nh][1][0], bfr[r][nh][1][1]);
+            const float2 cs2 = *reinterpret_cast<const float2*>(csum + 16 * r + 8 * nh + 2 * q4);
+            pk[nh][0] = pack_bf16x2(__fmaf_rn(sv[0], acc[0], zv[0] * cs2.x), __fmaf_rn(sv[0], acc[1], zv[0] * cs2.y));
+            pk[nh][1] = pack_bf16x2(__fmaf_rn(sv[1], acc[2], zv[1] * cs2.x), __fmaf_rn(sv[1], acc[3], zv[1] * cs2.y));
+          }
+        } else {
+          // keys: record (channel c) holds the unit's 32 tokens; y = s_c q + z_c
+          float sc[4], zc[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int c = 16 * r + 4 * q4 + m;
+            sc[m] = __half2float(__ushort_as_half(sbuf[c])) * kscale;
+            zc[m] = __half2float(__ushort_as_half(zbuf[c])) * kscale;
+          }
+          uint32_t ahi[4], alo[4];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int t = 16 * tt + g4 + 8 * half;
+            float y[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const int c = 16 * r + 4 * q4 + m;
+              const uint32_t q = bits_at(cbuf, c * 32 * BITS + t * BITS) & M;
+              y[m] = __fmaf_rn(sc[m], (float)q, zc[m]);
+            }
+            f16_split2(y[0], y[1], ahi[half], alo[half]);
+            f16_split2(y[2], y[3], ahi[2 + half], alo[2 + half]);
+          }
+#pragma unroll
+          for (int nh = 0; nh < 2; ++nh) {
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            mma_f16(acc, alo, bfr[r][nh][0][0], bfr[r][nh][0][1]);
+            mma_f16(acc, ahi, bfr[r][nh][1][0], bfr[r][nh][1][1]);
+            mma_f16(acc, ahi, bfr[r][nh][0][0], bfr[r][nh][0][1]);
+            pk[nh][0] = pack_bf16x2(acc[0] * kunscale, acc[1] * kunscale);
+            pk[nh][1] = pack_bf16x2(acc[2] * kunscale, acc[3] * kunscale);
+          }
+        }
+        // tiles (rows 0-7 | 8-15 of this 16-token tile) x (cols 16r .. +7 | 16r+8 .. +15)
+        stmatrix_x4(st_addr + 16 * tt * kPitch + 32 * r, pk[0][0], pk[0][1], pk[1][0], pk[1][1]);
+      }
+    }
+    __syncwarp();
+    // 32 rows of 256 B, contiguous in the output: each instruction writes two whole rows
+    uint16_t* obase = a.kv_out + (slice * a.k.T + 32LL * tgroup) * D;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int row = 2 * k + (lane >> 4), ch = lane & 15;
+      reinterpret_cast<uint4*>(obase + row * D)[ch] = *reinterpret_cast<const uint4*>(stg + row * kPitch + ch * 16);
+    }
+    __syncwarp();
+  }
+}
+
+namespace {
+constexpr int kSmem = kWarps * kWarpSmem;
+template <int BITS>
+cudaError_t kd_launch(const CodecArgs& a, int num_sms, cudaStream_t st) {
+  auto kern = kivi_decode_g16_kernel<BITS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
+  const long long units = a.k.slices() * (a.nt / 32);
+  const long long want = (units + kWarps - 1) / kWarps;
+  const int grid = (int)(want < num_sms ? want : num_sms);
+  kern<<<grid, kWarps * 32, kSmem, st>>>(a);
+  return cudaGetLastError();
+}
+}  // namespace
+
+bool kivi_decode_g16_supported(const CodecArgs& a) { return a.kivi && a.g == 16 && a.k.d == 128; }
+
+cudaError_t launch_kivi_decode_g16(const CodecArgs& a, int num_sms, cudaStream_t st) {
+  if (a.nt == 0) return cudaSuccess;
+  switch (a.bits) {
+    case 2: return kd_launch<2>(a, num_sms, st);
+    case 3: return kd_launch<3>(a, num_sms, st);
+    case 4: return kd_launch<4>(a, num_sms, st);
+    case 6: return kd_launch<6>(a, num_sms, st);
+    case 8: return kd_launch<8>(a, num_sms, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace cg
