@@ -104,6 +104,23 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings over all ranks of the process group
+    (the values unchanged on a single process).  Every rank must call it, in the same
+    order, with as many values."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_gbs(world_size, bytes_per_rank, ms):
+    """Whole-job throughput: the bytes all ranks processed over the slowest rank's time."""
+    return world_size * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 def run_cg(args):
     import torch
     import torch.distributed as dist
@@ -196,11 +213,8 @@ def run_cg(args):
     e2e_ms = s0.elapsed_time(s1) / e2e_steps if e2e_steps else float("nan")
 
     # --- max over ranks -----------------------------------------------------------------------
-    vals = torch.tensor([total_ms, statistics.mean(enc_ms), statistics.mean(dec_ms), e2e_ms], dtype=torch.float64,
-                        device=dev)
-    if ws > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, enc_avg, dec_avg, e2e_ms = [float(v) for v in vals.cpu()]
+    total_ms, enc_avg, dec_avg, e2e_ms = max_over_ranks(
+        [total_ms, statistics.mean(enc_ms), statistics.mean(dec_ms), e2e_ms], dev)
     if ws > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -216,7 +230,7 @@ def run_cg(args):
     dom_ms = max(enc_avg, dec_avg)
     achieved = alg_bytes / (dom_ms * 1e-3) / 1e9
     traffic = _traffic_record(dominant, args.bits)
-    value = ws * kv_bytes / (ms_step * 1e-3) / 1e9
+    value = job_gbs(ws, kv_bytes, ms_step)
     line = {
         "metric": "KV GB/s for fused gauge+quant encode/decode at %d bits; %% of HBM roofline" % args.bits,
         "value": round(value, 2),
@@ -241,7 +255,7 @@ def run_cg(args):
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": hbm_peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "traffic": traffic, "alg_bytes_per_value": bpv},
-        "e2e": None if args.no_e2e else {"value": round(ws * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": None if args.no_e2e else {"value": round(job_gbs(ws, kv_bytes, e2e_ms), 2), "unit": "GB/s",
                                          "h2d_bytes_per_step": kv_bytes, "d2h_bytes_per_step": kv_bytes},
         "gpu_launches": 2 * args.steps,
         "rows": rows,
