@@ -35,7 +35,8 @@ constexpr int kTile = 128;      // tokens per tile
 constexpr int kD = 128;         // d_head of this kernel
 constexpr int kOpBytes = kTile * kD * 2;  // one bf16 128 x 128 operand: 32 KB
 constexpr int kSPitch = 129;    // fp32 pitch of the 128 x 128 staging matrix
-constexpr int kSpecThreads = 5 * 32;
+constexpr int kWorkers = 256;  // 8 worker warps; warp 8 issues the MMAs
+constexpr int kSpecThreads = kWorkers + 32;
 
 // K-major, 128-byte swizzle (rows of 128 B; 8-row atoms 1024 B apart)
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t addr) {
@@ -122,7 +123,7 @@ struct SpecSmem {
   uint64_t* bars;      // a_full, t_full, d_full, t2_full
   uint32_t* tmem_base;
 };
-constexpr int kSpecSmem = 1024 + 5 * kOpBytes + kTile * kSPitch * 4 + (256 + 16 + 8) * 4 + 4 * 8 + 16;
+constexpr int kSpecSmem = 1024 + 5 * kOpBytes + kTile * kSPitch * 4 + (256 + 32 + 8) * 4 + 4 * 8 + 16;
 
 __device__ inline SpecSmem spec_carve(unsigned char* raw) {
   SpecSmem s;
@@ -136,7 +137,7 @@ __device__ inline SpecSmem spec_carve(unsigned char* raw) {
   s.Gs = s.S;
   s.C16 = s.S + kTile * kSPitch;
   s.red = s.C16 + 256;
-  s.blk = s.red + 16;
+  s.blk = s.red + 32;
   s.bars = reinterpret_cast<uint64_t*>(s.blk + 8);
   s.tmem_base = reinterpret_cast<uint32_t*>(s.bars + 4);
   return s;
@@ -173,9 +174,9 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
   }
   for (int e = tid; e < 256; e += kSpecThreads) sm.C16[e] = dct_coef(e / 16, e % 16, 16);
   if (tid == 0) {
-    mbar_init(a_full, 4);
+    mbar_init(a_full, kWorkers / 32);
     mbar_init(t_full, 1);
-    mbar_init(d_full, 4);
+    mbar_init(d_full, kWorkers / 32);
     mbar_init(t2_full, 1);
     fence_mbar_init();
   }
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
     for (int tile = 0; tile < tiles; ++tile, ++it) {
       const uint32_t ph = (uint32_t)(it & 1);
       const long long row0 = slice * a.k.T + (long long)tile * kTile;
-      if (warp == 4) {
+      if (warp == kWorkers / 32) {
         // ---------------- MMA issue ----------------
         if (lane == 0) {
           mbar_wait(a_full, ph, a.status);
@@ -250,49 +251,51 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
       }
       // ---------------- A: X' row = G x, split into the bf16 operand ----------------
       if (a.has_g) {  // G of this slice, staged in the (idle) U1 buffer
-        for (int e = tid; e < 2048; e += 128) sm.Gs[e] = Gp[e];
-        named_bar_sync(1, 128);
+        for (int e = tid; e < 2048; e += kWorkers) sm.Gs[e] = Gp[e];
+        named_bar_sync(1, kWorkers);
       }
       {
-        const int t = tid;
-        float x[128];
+        const int t = tid & 127, hf = tid >> 7;  // token row, channel half 64 hf .. 64 hf + 63
+        float x[64];
         if (a.x_fp32) {
-          const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.x) + (row0 + t) * kD);
+          const float4* src =
+              reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.x) + (row0 + t) * kD + 64 * hf);
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
+          for (int q = 0; q < 16; ++q) {
             const float4 v = src[q];
             x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
           }
         } else {
-          const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.x) + (row0 + t) * kD);
+          const uint4* src =
+              reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.x) + (row0 + t) * kD + 64 * hf);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
+          for (int q = 0; q < 8; ++q) {
             const uint4 w = src[q];
             x[8 * q + 0] = bf16lo(w.x); x[8 * q + 1] = bf16hi(w.x); x[8 * q + 2] = bf16lo(w.y); x[8 * q + 3] = bf16hi(w.y);
             x[8 * q + 4] = bf16lo(w.z); x[8 * q + 5] = bf16hi(w.z); x[8 * q + 6] = bf16lo(w.w); x[8 * q + 7] = bf16hi(w.w);
           }
         }
 #pragma unroll
-        for (int cb = 0; cb < 16; ++cb) {  // 8 channels per 16-byte chunk
+        for (int cb = 0; cb < 8; ++cb) {  // 8 channels per 16-byte chunk
           float y8[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int c = 8 * cb + e;
+            const int cl = 8 * cb + e, c = 64 * hf + cl;  // local and head channel
             if (a.has_g) {
-              const int r = c >> 4, i = c & 15;
+              const int rl = cl >> 4, r = c >> 4, i = c & 15;
               const float4* gi = reinterpret_cast<const float4*>(sm.Gs + (r * 16 + i) * 16);
               float acc = 0.0f;
 #pragma unroll
               for (int j4 = 0; j4 < 4; ++j4) {
                 const float4 g = gi[j4];
-                acc = __fmaf_rn(g.x, x[16 * r + 4 * j4], acc);
-                acc = __fmaf_rn(g.y, x[16 * r + 4 * j4 + 1], acc);
-                acc = __fmaf_rn(g.z, x[16 * r + 4 * j4 + 2], acc);
-                acc = __fmaf_rn(g.w, x[16 * r + 4 * j4 + 3], acc);
+                acc = __fmaf_rn(g.x, x[16 * rl + 4 * j4], acc);
+                acc = __fmaf_rn(g.y, x[16 * rl + 4 * j4 + 1], acc);
+                acc = __fmaf_rn(g.z, x[16 * rl + 4 * j4 + 2], acc);
+                acc = __fmaf_rn(g.w, x[16 * rl + 4 * j4 + 3], acc);
               }
               y8[e] = acc;
             } else {
-              y8[e] = x[c];
+              y8[e] = x[cl];
             }
           }
           uint32_t hw[4], lw[4];
@@ -302,34 +305,36 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
             hw[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
             lw[e] = (uint32_t)bf16_rn(y8[2 * e] - bf16_f(h0)) | ((uint32_t)bf16_rn(y8[2 * e + 1] - bf16_f(h1)) << 16);
           }
-          *reinterpret_cast<uint4*>(sm.ahi + swz(t, 8 * cb)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(sm.alo + swz(t, 8 * cb)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          *reinterpret_cast<uint4*>(sm.ahi + swz(t, 64 * hf + 8 * cb)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(sm.alo + swz(t, 64 * hf + 8 * cb)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(a_full);
       }
-      if (a.has_g) named_bar_sync(1, 128);  // all rows gauged before U1 overwrites the staged G
+      if (a.has_g) named_bar_sync(1, kWorkers);  // all rows gauged before U1 overwrites the staged G
       // ---------------- C: U1 rows to shared memory, token DCT and block statistics ----------------
       mbar_wait(t_full, ph, a.status);
       fence_after();
       {
-        const int t = tid;
+        const int t = 32 * (warp & 3) + lane, ch = warp >> 2;  // TMEM lane quarter of this warp, column half
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int c4 = 2 * ch + c2;
           float v[32];
-          ld32(tmem + 32 * c4 + ((uint32_t)(32 * warp) << 16), v);
+          ld32(tmem + 32 * c4 + ((uint32_t)(32 * (warp & 3)) << 16), v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) sm.S[t * kSPitch + 32 * c4 + j] = v[j];
         }
       }
       fence_before();
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kWorkers);
       {
-        const int v = tid;  // channel-frequency column
-        const int obase = (int)(row0 / 16);  // first block index of this tile
+        const int v = tid & 127, bh = tid >> 7;  // channel-frequency column, half of the tile's blocks
+        const int obase = (int)(row0 / 16);       // first block index of this tile
         const float inv_tau = 1.0f / a.tau;
-        for (int kb = 0; kb < kTile / 16; ++kb) {
+        float* red = sm.red + 12 * bh;
+        for (int kb = 4 * bh; kb < 4 * bh + 4; ++kb) {
           float col[16], U[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) col[t] = sm.S[(16 * kb + t) * kSPitch + v];
@@ -372,16 +377,16 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
             r_sum += __shfl_xor_sync(0xffffffffu, r_sum, o);
           }
           if (lane == 0) {
-            sm.red[warp * 3 + 0] = e_sum;
-            sm.red[warp * 3 + 1] = f_sum;
-            sm.red[warp * 3 + 2] = r_sum;
+            red[(warp & 3) * 3 + 0] = e_sum;
+            red[(warp & 3) * 3 + 1] = f_sum;
+            red[(warp & 3) * 3 + 2] = r_sum;
           }
-          named_bar_sync(1, 128);
-          const float E = (sm.red[0] + sm.red[3]) + (sm.red[6] + sm.red[9]);
-          const float F = (sm.red[1] + sm.red[4]) + (sm.red[7] + sm.red[10]);
-          const float R = (sm.red[2] + sm.red[5]) + (sm.red[8] + sm.red[11]);
+          named_bar_sync(2 + bh, 128);
+          const float E = (red[0] + red[3]) + (red[6] + red[9]);
+          const float F = (red[1] + red[4]) + (red[7] + red[10]);
+          const float R = (red[2] + red[5]) + (red[8] + red[11]);
           const float lf = E > 0.0f ? F / E : 0.0f;
-          if (tid == 0) {
+          if (v == 0) {
             a.lfreq[obase + kb] = lf;
             a.lrate[obase + kb] = R / (16.0f * kD);
           }
@@ -413,7 +418,7 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
               *reinterpret_cast<uint16_t*>(sm.alo + swz(16 * kb + 15 - t, v)) = bf16_rn(d1 - bf16_f(h1));
             }
           }
-          named_bar_sync(1, 128);  // sm.red reused by the next block
+          named_bar_sync(2 + bh, 128);  // red reused by the next block
         }
       }
       if (!a.want_grad) continue;
@@ -424,10 +429,10 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
       mbar_wait(t2_full, ph, a.status);
       fence_after();
       {
-        const int c = tid, r = c >> 4;
-        for (int c4 = 0; c4 < 4; ++c4) {
+        const int c = tid & 127, r = c >> 4, th = tid >> 7;  // channel (= TMEM lane), token half
+        for (int c4 = 2 * th; c4 < 2 * th + 2; ++c4) {
           float v[32];
-          ld32(tmem + 128 + 32 * c4 + ((uint32_t)(32 * warp) << 16), v);  // dX'^T row c: tokens 32 c4 ..
+          ld32(tmem + 128 + 32 * c4 + ((uint32_t)(32 * (warp & 3)) << 16), v);  // dX'^T row c: tokens 32 c4 ..
 #pragma unroll 8
           for (int tt = 0; tt < 32; ++tt) {
             const long long row = row0 + 32 * c4 + tt;
@@ -455,12 +460,24 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
         }
       }
       fence_before();
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kWorkers);
     }
-    if (warp < 4 && a.want_grad) {
-      float4* dst = reinterpret_cast<float4*>(a.dg_part + slice * (long long)kD * 16 + tid * 16);
+    if (warp < kWorkers / 32 && a.want_grad) {  // the two token halves' partials of channel c, in a fixed order
+      const int c = tid & 127;
+      float* part = sm.S + c * 16;  // U1 staging is free here
+      if (tid >= 128) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = make_float4(dg[4 * q], dg[4 * q + 1], dg[4 * q + 2], dg[4 * q + 3]);
+        for (int j = 0; j < 16; ++j) part[j] = dg[j];
+      }
+      named_bar_sync(1, kWorkers);
+      if (tid < 128) {
+        float4* dst = reinterpret_cast<float4*>(a.dg_part + slice * (long long)kD * 16 + c * 16);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_float4(dg[4 * q] + part[4 * q], dg[4 * q + 1] + part[4 * q + 1], dg[4 * q + 2] + part[4 * q + 2],
+                               dg[4 * q + 3] + part[4 * q + 3]);
+      }
+      named_bar_sync(1, kWorkers);  // the staging is written by the next slice's first tile
     }
   }
   fence_before();
