@@ -313,7 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // B = G^T (bf16, swizzled K-major, column sums of the same bf16 values kept
 // beside it); the same warps then read the accumulator and write bf16.
 namespace {
-constexpr int kDecThreads = (kEpiWarps + 2) * 32;
+constexpr int kDecEpi = 8;  // two warpgroups taking alternate blocks: code expansion, then epilogue
+constexpr int kDecThreads = (kDecEpi + 2) * 32;
 struct FdSmem {
   unsigned char* as;  // 2 x 32 KB A tiles
   unsigned char* gs;  // 2 x 32 KB G^T tiles
@@ -370,14 +371,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.a_full[s], kEpiWarps);
+      mbar_init(&sm.a_full[s], 4);  // the warpgroup that takes the block
       mbar_init(&sm.a_empty[s], 1);
       mbar_init(&sm.g_full[s], 1);
       // released by the tensor cores (done reading G^T) and by the epilogue
       // warps (done reading the column sums)
-      mbar_init(&sm.g_empty[s], 1 + kEpiWarps);
+      mbar_init(&sm.g_empty[s], 1 + kDecEpi);
       mbar_init(&sm.t_full[s], 1);
-      mbar_init(&sm.t_empty[s], kEpiWarps);
+      mbar_init(&sm.t_empty[s], 4);
     }
     fence_mbar_init();
   }
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_base;
 
-  if (warp == kEpiWarps) {
+  if (warp == kDecEpi) {
     // ---------------- G^T staging (bf16, swizzled, rows = outputs n) and column sums ----------------
     long long slice = b0 / bps;
     int bq = (int)(b0 - slice * bps);
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
         ++slice;
       }
     }
-  } else if (warp == kEpiWarps + 1) {
+  } else if (warp == kDecEpi + 1) {
     // ---------------- MMA issue ----------------
     if (lane == 0) {
       long long slice = b0 / bps;
@@ -460,95 +461,90 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
       }
     }
   } else {
-    // ---------------- code expansion (block i+1) and epilogue (block i); thread = token row ----------------
-    const int row = 32 * warp + lane;
-    long long slice_c = b0 / bps;  // cursor of the block being expanded
-    int bq_c = (int)(b0 - slice_c * bps);
-    long long slice_e = slice_c;   // cursor of the block in the epilogue
-    int bq_e = bq_c;
-    int gcount_e = 0;
-    auto expand = [&](int i) {
-      const int ab = i & 1;
-      mbar_wait(&sm.a_empty[ab], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.status);
-      const int valid = min(128, a.nt - 128 * bq_c);
-      const int tok = a.t0 + 128 * bq_c + min(row, valid - 1);  // rows past the range repeat a valid row
-      const uint4* src = reinterpret_cast<const uint4*>(a.codes_in + slice_c * slice_code_bytes +
-                                                        (long long)(tok / 16) * (16 * D * BITS / 8) +
-                                                        (tok % 16) * (D * BITS / 8));
-      uint32_t words[4 * BITS + 1];
-#pragma unroll
-      for (int w = 0; w < BITS; ++w) {
-        const uint4 v = src[w];
-        words[4 * w] = v.x; words[4 * w + 1] = v.y; words[4 * w + 2] = v.z; words[4 * w + 3] = v.w;
-      }
-      words[4 * BITS] = 0;
-      unsigned char* adst = sm.as + ab * kBlockBytes;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {  // 16-byte chunk c = channels 8c .. 8c+7
-        uint32_t q[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int bit = (8 * c + e) * BITS;
-          q[e] = __funnelshift_r(words[bit >> 5], words[(bit >> 5) + 1], bit & 31) & M;
-        }
-        const uint4 w = make_uint4(code_pair_bf16(q[0], q[1]), code_pair_bf16(q[2], q[3]), code_pair_bf16(q[4], q[5]),
-                                   code_pair_bf16(q[6], q[7]));
-        *reinterpret_cast<uint4*>(adst + sw128_offset(row, 8 * c)) = w;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.a_full[ab]);
-      if (++bq_c == bps) {
-        bq_c = 0;
-        ++slice_c;
-      }
-    };
-    if (n_blocks > 0) expand(0);
+    // ---------------- warpgroup wg takes blocks i = wg, wg + 2, ...: code expansion, then epilogue;
+    // thread = token row (the other warpgroup's work covers this block's MMA) ----------------
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int row = 32 * quarter + lane;
+    long long slice = b0 / bps;
+    int bq = (int)(b0 - slice * bps);
+    int gcount = 0;
     for (int i = 0; i < n_blocks; ++i) {
-      if (i + 1 < n_blocks) expand(i + 1);
-      const int ab = i & 1;
-      const int gb = gcount_e & 1;
-      const int valid = min(128, a.nt - 128 * bq_e);
-      const int tok = a.t0 + 128 * bq_e + row;
-      float sf = 0.0f, zf = 0.0f;
-      if (row < valid) {
-        const long long bidx = slice_e * (a.k.T / 16) + tok / 16;
-        sf = __half2float(__ushort_as_half(__ldg(a.scales_in + bidx)));
-        zf = __half2float(__ushort_as_half(__ldg(a.zeros_in + bidx)));
-      }
-      mbar_wait(&sm.t_full[ab], (uint32_t)(i >> 1) & 1u, a.status);
-      tc_fence_after();
-      const uint32_t taddr = tmem + ab * 128 + ((uint32_t)(32 * warp) << 16);
-      const float* cs = sm.colsum + gb * 128;
-      uint4* dst = reinterpret_cast<uint4*>(a.kv_out + (slice_e * a.k.T + tok) * (long long)D);
+      const int gb = gcount & 1;
+      const bool last_of_slice = (bq + 1 == bps) || (i + 1 == n_blocks);
+      if ((i & 1) == wg) {
+        const int ab = i & 1;  // == wg: each warpgroup has its own A buffer and accumulator
+        const int valid = min(128, a.nt - 128 * bq);
+        {  // codes of the block -> exact bf16 integers, swizzled K-major A operand
+          mbar_wait(&sm.a_empty[ab], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.status);
+          const int tok = a.t0 + 128 * bq + min(row, valid - 1);  // rows past the range repeat a valid row
+          const uint4* src = reinterpret_cast<const uint4*>(a.codes_in + slice * slice_code_bytes +
+                                                            (long long)(tok / 16) * (16 * D * BITS / 8) +
+                                                            (tok % 16) * (D * BITS / 8));
+          uint32_t words[4 * BITS + 1];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float v[32];
-        tmem_ld32(taddr + 32 * c4, v);
-        tmem_wait_ld();
+          for (int w = 0; w < BITS; ++w) {
+            const uint4 v = src[w];
+            words[4 * w] = v.x; words[4 * w + 1] = v.y; words[4 * w + 2] = v.z; words[4 * w + 3] = v.w;
+          }
+          words[4 * BITS] = 0;
+          unsigned char* adst = sm.as + ab * kBlockBytes;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {  // 16-byte chunk c = channels 8c .. 8c+7
+            uint32_t q[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int bit = (8 * c + e) * BITS;
+              q[e] = __funnelshift_r(words[bit >> 5], words[(bit >> 5) + 1], bit & 31) & M;
+            }
+            const uint4 w = make_uint4(code_pair_bf16(q[0], q[1]), code_pair_bf16(q[2], q[3]),
+                                       code_pair_bf16(q[4], q[5]), code_pair_bf16(q[6], q[7]));
+            *reinterpret_cast<uint4*>(adst + sw128_offset(row, 8 * c)) = w;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.a_full[ab]);
+        }
+        const int tok = a.t0 + 128 * bq + row;
+        float sf = 0.0f, zf = 0.0f;
         if (row < valid) {
+          const long long bidx = slice * (a.k.T / 16) + tok / 16;
+          sf = __half2float(__ushort_as_half(__ldg(a.scales_in + bidx)));
+          zf = __half2float(__ushort_as_half(__ldg(a.zeros_in + bidx)));
+        }
+        mbar_wait(&sm.t_full[ab], (uint32_t)(i >> 1) & 1u, a.status);
+        tc_fence_after();
+        const uint32_t taddr = tmem + ab * 128 + ((uint32_t)(32 * quarter) << 16);
+        const float* cs = sm.colsum + gb * 128;
+        uint4* dst = reinterpret_cast<uint4*>(a.kv_out + (slice * a.k.T + tok) * (long long)D);
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            uint4 o;
-            o.x = pack_bf16x2(__fmaf_rn(sf, v[j + 0], zf * cs[32 * c4 + j + 0]), __fmaf_rn(sf, v[j + 1], zf * cs[32 * c4 + j + 1]));
-            o.y = pack_bf16x2(__fmaf_rn(sf, v[j + 2], zf * cs[32 * c4 + j + 2]), __fmaf_rn(sf, v[j + 3], zf * cs[32 * c4 + j + 3]));
-            o.z = pack_bf16x2(__fmaf_rn(sf, v[j + 4], zf * cs[32 * c4 + j + 4]), __fmaf_rn(sf, v[j + 5], zf * cs[32 * c4 + j + 5]));
-            o.w = pack_bf16x2(__fmaf_rn(sf, v[j + 6], zf * cs[32 * c4 + j + 6]), __fmaf_rn(sf, v[j + 7], zf * cs[32 * c4 + j + 7]));
-            dst[(32 * c4 + j) / 8] = o;
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float v[32];
+          tmem_ld32(taddr + 32 * c4, v);
+          tmem_wait_ld();
+          if (row < valid) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 o;
+              o.x = pack_bf16x2(__fmaf_rn(sf, v[j + 0], zf * cs[32 * c4 + j + 0]), __fmaf_rn(sf, v[j + 1], zf * cs[32 * c4 + j + 1]));
+              o.y = pack_bf16x2(__fmaf_rn(sf, v[j + 2], zf * cs[32 * c4 + j + 2]), __fmaf_rn(sf, v[j + 3], zf * cs[32 * c4 + j + 3]));
+              o.z = pack_bf16x2(__fmaf_rn(sf, v[j + 4], zf * cs[32 * c4 + j + 4]), __fmaf_rn(sf, v[j + 5], zf * cs[32 * c4 + j + 5]));
+              o.w = pack_bf16x2(__fmaf_rn(sf, v[j + 6], zf * cs[32 * c4 + j + 6]), __fmaf_rn(sf, v[j + 7], zf * cs[32 * c4 + j + 7]));
+              dst[(32 * c4 + j) / 8] = o;
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.t_empty[ab]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.t_empty[ab]);
-      const bool last_of_slice = (bq_e + 1 == bps) || (i + 1 == n_blocks);
-      if (last_of_slice) {
+      if (last_of_slice) {  // every epilogue warp is past this slice: its G^T and column sums may go
+        __syncwarp();
         if (lane == 0) mbar_arrive(&sm.g_empty[gb]);
-        ++gcount_e;
+        ++gcount;
       }
-      if (++bq_e == bps) {
-        bq_e = 0;
-        ++slice_e;
+      if (++bq == bps) {
+        bq = 0;
+        ++slice;
       }
     }
   }
