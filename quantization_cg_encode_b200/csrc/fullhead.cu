@@ -26,10 +26,12 @@ namespace cg {
 
 namespace {
 
-constexpr int kXStages = 3;
+constexpr int kXStages = 4;
 constexpr int kBlockBytes = 128 * 128 * 2;  // 32 KB of bf16
-constexpr int kEpiWarps = 4;
-constexpr int kThreads = (kEpiWarps + 2) * 32;  // 4 epilogue, 1 TMA / G, 1 MMA
+// encoder: three epilogue warpgroups taking blocks in turn, four TMEM accumulators
+constexpr int kEncGroups = 3;
+constexpr int kEncEpi = 4 * kEncGroups;
+constexpr int kThreads = (kEncEpi + 2) * 32;  // 12 epilogue, 1 TMA / G, 1 MMA
 // tcgen05 instruction descriptor: D fp32, A and B bf16, both K-major, N = 128, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
@@ -104,16 +106,33 @@ __device__ inline FhSmem fh_carve(unsigned char* raw) {
   s.g_full = bars + 2 * kXStages;
   s.g_empty = s.g_full + 2;
   s.t_full = s.g_empty + 2;
-  s.t_empty = s.t_full + 2;
-  s.tmem_base = reinterpret_cast<uint32_t*>(s.t_empty + 2);
+  s.t_empty = s.t_full + 4;
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.t_empty + 4);
   return s;
 }
-constexpr int kFhSmem = 1024 + (kXStages + 2) * kBlockBytes + (2 * kXStages + 6) * 8 + 16;
+constexpr int kFhSmem = 1024 + (kXStages + 2) * kBlockBytes + (2 * kXStages + 12) * 8 + 16;
+
+// The BITS words of 32 packed codes at p (4 * BITS bytes; p is aligned to 16 bytes for
+// BITS = 4 and 8, to 8 for BITS = 2 and 6, to 4 for BITS = 3).
+template <int BITS>
+__device__ __forceinline__ void store_code_words(unsigned char* p, const uint32_t (&w)[BITS]) {
+  if constexpr (BITS % 4 == 0) {
+#pragma unroll
+    for (int k = 0; k < BITS / 4; ++k)
+      reinterpret_cast<uint4*>(p)[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  } else if constexpr (BITS % 2 == 0) {
+#pragma unroll
+    for (int k = 0; k < BITS / 2; ++k) reinterpret_cast<uint2*>(p)[k] = make_uint2(w[2 * k], w[2 * k + 1]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) reinterpret_cast<uint32_t*>(p)[k] = w[k];
+  }
+}
 
 }  // namespace
 
 template <int BITS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps registers at 128 (4 warps per scheduler)
     fullhead_encode_kernel(const __grid_constant__ CUtensorMap tmap, CodecArgs a) {
   constexpr int D = 128;
   constexpr int QMAX = (1 << BITS) - 1;
@@ -134,14 +153,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.g_full[s], 1);
       mbar_init(&sm.g_empty[s], 1);
+    }
+    for (int s = 0; s < 4; ++s) {
       mbar_init(&sm.t_full[s], 1);
-      mbar_init(&sm.t_empty[s], kEpiWarps);
+      mbar_init(&sm.t_empty[s], 4);  // the four warps of the warpgroup that took the block
     }
     fence_mbar_init();
   }
-  if (warp == 0) {  // TMEM: two 128-column fp32 accumulators
+  if (warp == 0) {  // TMEM: four 128-column fp32 accumulators
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(sm.tmem_base)),
-                 "r"(256));
+                 "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -149,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_base;
 
-  if (warp == kEpiWarps) {
+  if (warp == kEncEpi) {
     // ---------------- TMA x blocks + G staging ----------------
     long long slice = b0 / bps;
     int bq = (int)(b0 - slice * bps);
@@ -191,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++slice;
       }
     }
-  } else if (warp == kEpiWarps + 1) {
+  } else if (warp == kEncEpi + 1) {
     // ---------------- MMA issue (one thread) ----------------
     if (lane == 0) {
       long long slice = b0 / bps;
@@ -200,9 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < n_blocks; ++i) {
         const int gb = gcount & 1;
         if (i == 0 || bq == 0) mbar_wait(&sm.g_full[gb], (uint32_t)(gcount >> 1) & 1u, a.status);
-        const int s = i % kXStages, acc = i & 1;
+        const int s = i % kXStages, acc = i & 3;
         mbar_wait(&sm.x_full[s], (uint32_t)(i / kXStages) & 1u, a.status);
-        mbar_wait(&sm.t_empty[acc], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.status);
+        mbar_wait(&sm.t_empty[acc], ((uint32_t)(i >> 2) & 1u) ^ 1u, a.status);
         tc_fence_after();
         const uint32_t xa = smem_u32(sm.xs + s * kBlockBytes), ga = smem_u32(sm.gs + gb * kBlockBytes);
 #pragma unroll
@@ -224,68 +245,77 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue: thread = token row of the block ----------------
-    const int row = 32 * warp + lane;
+    // ---------------- epilogue: warpgroup wg takes blocks i with i % 3 == wg; thread = token row ----------------
+    const int wg = warp >> 2, quarter = warp & 3;
+    const int row = 32 * quarter + lane;
     const double inv_qmax = 1.0 / (double)QMAX;
     const long long slice_code_bytes = (long long)a.k.T * D * BITS / 8;
     long long slice = b0 / bps;
     int bq = (int)(b0 - slice * bps);
     for (int i = 0; i < n_blocks; ++i) {
-      const int acc = i & 1;
-      mbar_wait(&sm.t_full[acc], (uint32_t)(i >> 1) & 1u, a.status);
-      tc_fence_after();
-      float y[128];
-      const uint32_t taddr = tmem + acc * 128 + ((uint32_t)(32 * warp) << 16);
+      if (i % kEncGroups == wg) {
+        const int acc = i & 3;
+        mbar_wait(&sm.t_full[acc], (uint32_t)(i >> 2) & 1u, a.status);
+        tc_fence_after();
+        const uint32_t taddr = tmem + acc * 128 + ((uint32_t)(32 * quarter) << 16);
+        const int valid = min(128, a.nt - 128 * bq);
+        const int tok = a.t0 + 128 * bq + row;
+        // pass 1: the row's range, then the 16-token block's (16 lanes)
+        float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(taddr + 32 * c, v);
+          tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(taddr + 32 * c, v);
+          for (int j = 0; j < 32; ++j) {
+            mn = fminf(mn, v[j]);
+            mx = fmaxf(mx, v[j]);
+          }
+        }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) y[32 * c + j] = v[j];
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.t_empty[acc]);
-
-      const int valid = min(128, a.nt - 128 * bq);
-      const int tok = a.t0 + 128 * bq + row;
-      // range of the 16-token block: this row's 128 values, then 16 lanes
-      float mn = y[0], mx = y[0];
-#pragma unroll
-      for (int j = 1; j < 128; ++j) {
-        mn = fminf(mn, y[j]);
-        mx = fmaxf(mx, y[j]);
-      }
-#pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
-      if (row < valid) {
+        for (int o = 8; o >= 1; o >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
         const QParams qp = quant_params(mn, mx, inv_qmax);
-        if (a.gauged) {
-          float4* gd = reinterpret_cast<float4*>(a.gauged + (slice * a.k.T + tok) * D);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) gd[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
-        }
-        // token row's 128 codes: bytes [r16 * 16 * BITS, +16 * BITS) of its block's record
-        uint32_t words[4 * BITS];
-#pragma unroll
-        for (int w = 0; w < 4 * BITS; ++w) words[w] = 0;
-#pragma unroll
-        for (int j = 0; j < 128; ++j) {
-          const uint32_t q = quantize_one(y[j], qp.zf, qp.inv, QMAX);
-          const int bit = j * BITS;
-          words[bit >> 5] |= q << (bit & 31);
-          if ((bit & 31) + BITS > 32) words[(bit >> 5) + 1] |= q >> (32 - (bit & 31));
-        }
+        // pass 2: codes of the row, 32 at a time (BITS packed words each, little-endian),
+        // stored as they are made: the row's codes are bytes [r16 * 16 * BITS, +16 * BITS)
+        // of its 16-token block's record
         const int tile = tok / 16, r16 = tok % 16;
-        uint4* dst = reinterpret_cast<uint4*>(a.codes + slice * slice_code_bytes + (long long)tile * (16 * D * BITS / 8) +
-                                              r16 * (D * BITS / 8));
+        unsigned char* dst = a.codes + slice * slice_code_bytes + (long long)tile * (16 * D * BITS / 8) +
+                             r16 * (D * BITS / 8);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float v[32];
+          tmem_ld32(taddr + 32 * c, v);
+          tmem_wait_ld();
+          if (c == 3) {  // the accumulator is free once the last columns are in registers
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.t_empty[acc]);
+          }
+          if (a.gauged && row < valid) {
+            float4* gd = reinterpret_cast<float4*>(a.gauged + (slice * a.k.T + tok) * D + 32 * c);
 #pragma unroll
-        for (int w = 0; w < BITS; ++w) dst[w] = make_uint4(words[4 * w], words[4 * w + 1], words[4 * w + 2], words[4 * w + 3]);
-        if ((lane & 15) == 0) {
+            for (int j = 0; j < 8; ++j) gd[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          }
+          uint32_t words[BITS];
+#pragma unroll
+          for (int w = 0; w < BITS; ++w) words[w] = 0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            // q = clamp(rne(fl(fl(y - z) * inv)), 0, qmax): clamped first, then rounded (RNE)
+            // by adding 1.5 * 2^23, which leaves the integer in the low mantissa bits
+            const float t = fminf(fmaxf(__fmul_rn(__fsub_rn(v[j], qp.zf), qp.inv), 0.0f), (float)QMAX);
+            const uint32_t q = __float_as_uint(__fadd_rn(t, 12582912.0f)) & ((1u << BITS) - 1u);
+            const int bit = j * BITS;
+            words[bit >> 5] |= q << (bit & 31);
+            if ((bit & 31) + BITS > 32) words[(bit >> 5) + 1] |= q >> (32 - (bit & 31));
+          }
+          if (row < valid) store_code_words<BITS>(dst + c * 4 * BITS, words);
+        }
+        if (row < valid && (lane & 15) == 0) {
           const long long bidx = slice * (a.k.T / 16) + tile;
           a.scales[bidx] = qp.sh;
           a.zeros[bidx] = qp.zh;
@@ -301,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
 }
 
