@@ -8,10 +8,12 @@
 // before the backend and inverted after it, with explicit recovery.
 //
 // One warp owns a unit of 32 tokens x 32 channels of one head slice; lane t
-// holds token t's 32 gauged values (32 / g groups).  A key range is one channel
-// across the 32 lanes (redux.sync), a value range is one lane's 32 values.
-// Codes are packed across lanes with redux.sync.or: lane t contributes its code
-// at bits [t b, t b + b) of the range's little-endian bit stream.
+// holds token t's 32 gauged values (32 / g groups).  A value range is one
+// lane's 32 values.  For keys the encoder transposes the unit through shared
+// memory, so that lane c holds channel c's 32 tokens: a key range is then one
+// lane's values too, and lane c packs its record (token t's code at bits
+// [t b, t b + b) of the little-endian bit stream) by itself.  The decoder
+// gathers key codes across lanes with shuffles.
 // The gauged values are the same fp32 FMA chains (j = 0..g-1 from +0) as the
 // block-uniform encoder, so codes are bit-reproducible.
 #include "cg_kernels.cuh"
@@ -21,12 +23,6 @@ namespace cg {
 namespace {
 
 constexpr int kWarps = 8;
-
-__device__ __forceinline__ uint32_t warp_or(uint32_t v) {
-  uint32_t r;
-  asm volatile("redux.sync.or.b32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
-  return r;
-}
 
 struct KUnit {
   long long slice;
@@ -56,12 +52,21 @@ __device__ inline void load_gauge(float* Gs, const CodecArgs& a, long long slice
 
 }  // namespace
 
+// Shared memory of the encoder per warp: its staged gauge (32 G floats) and a
+// 32 x 33 fp32 transpose buffer (the padding keeps both directions free of
+// bank conflicts).
+template <int G>
+constexpr int kivi_encode_smem() {
+  return kWarps * (32 * G + 32 * 33) * 4;
+}
+
 template <int G, int BITS>
 __global__ void __launch_bounds__(kWarps * 32) kivi_encode_kernel(CodecArgs a) {
   constexpr int QMAX = (1 << BITS) - 1;
-  __shared__ __align__(16) float sG[kWarps][32 * G];
+  extern __shared__ __align__(16) float kivi_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* Gs = sG[warp];
+  float* Gs = kivi_smem + warp * 32 * G;
+  float* Ts = kivi_smem + kWarps * 32 * G + warp * 32 * 33;
   const long long units = a.k.slices() * (a.nt / 32) * (a.k.d / 32);
   const double inv_qmax = 1.0 / (double)QMAX;
   long long loaded = -1;
@@ -118,44 +123,41 @@ __global__ void __launch_bounds__(kWarps * 32) kivi_encode_kernel(CodecArgs a) {
     const long long slice_bytes = (long long)a.k.T * a.k.d * BITS / 8;
     const long long slice_ranges = (long long)a.k.T * a.k.d / 32;
     if (s == 0) {
-      // ---- keys: range per channel over the 32 tokens (lanes) ----
-      // lane c ends up with channel c's min / max
-      float cmn = 0.0f, cmx = 0.0f;
+      // ---- keys: range per channel over the 32 tokens; transpose so that lane c
+      // holds channel c ----
+      __syncwarp();  // the previous unit's reads of the buffer are done
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float mn = warp_min_f32(y[c]), mx = warp_max_f32(y[c]);
-        if (lane == c) {
-          cmn = mn;
-          cmx = mx;
-        }
+      for (int c = 0; c < 32; ++c) Ts[lane * 33 + c] = y[c];
+      __syncwarp();
+      float yc[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) yc[t] = Ts[t * 33 + lane];
+      float mn = yc[0], mx = yc[0];
+#pragma unroll
+      for (int t = 1; t < 32; ++t) {
+        mn = fminf(mn, yc[t]);
+        mx = fmaxf(mx, yc[t]);
       }
-      const QParams qp = quant_params(cmn, cmx, inv_qmax);
+      const QParams qp = quant_params(mn, mx, inv_qmax);
       const int tgroup = (a.t0 / 32) + ku.tg;
       const long long ridx = ku.slice * slice_ranges + (long long)tgroup * a.k.d + 32 * ku.cg + lane;
       a.scales[ridx] = qp.sh;
       a.zeros[ridx] = qp.zh;
       // codes: channel c's record = 32 codes, token-ascending; lane c stores record c
-      uint32_t mine[BITS];
+      uint32_t words[BITS];
 #pragma unroll
-      for (int w = 0; w < BITS; ++w) mine[w] = 0;
+      for (int w = 0; w < BITS; ++w) words[w] = 0;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float zf = __shfl_sync(0xffffffffu, qp.zf, c), inv = __shfl_sync(0xffffffffu, qp.inv, c);
-        const uint32_t q = quantize_one(y[c], zf, inv, QMAX);
-        const int bit = lane * BITS;  // position of this token's code in the 32 * BITS-bit record
-        const uint32_t lo = q << (bit & 31);
-        const uint32_t hi = (bit & 31) + BITS > 32 ? q >> (32 - (bit & 31)) : 0u;
-#pragma unroll
-        for (int w = 0; w < BITS; ++w) {
-          const uint32_t part = ((bit >> 5) == w ? lo : 0u) | ((bit >> 5) + 1 == w ? hi : 0u);
-          const uint32_t word = warp_or(part);
-          if (lane == c) mine[w] = word;
-        }
+      for (int t = 0; t < 32; ++t) {
+        const uint32_t q = quantize_one(yc[t], qp.zf, qp.inv, QMAX);
+        const int bit = t * BITS;
+        words[bit >> 5] |= q << (bit & 31);
+        if ((bit & 31) + BITS > 32) words[(bit >> 5) + 1] |= q >> (32 - (bit & 31));
       }
       uint32_t* rec = reinterpret_cast<uint32_t*>(a.codes + ku.slice * slice_bytes +
                                                    ((long long)tgroup * a.k.d + 32 * ku.cg + lane) * (4 * BITS));
 #pragma unroll
-      for (int w = 0; w < BITS; ++w) rec[w] = mine[w];
+      for (int w = 0; w < BITS; ++w) rec[w] = words[w];
     } else {
       // ---- values: range per token over its 32 channels (this lane) ----
       float mn = y[0], mx = y[0];
@@ -290,10 +292,15 @@ cudaError_t kivi_launch(const CodecArgs& a, bool encode, int num_sms, cudaStream
   const long long units = a.k.slices() * (a.nt / 32) * (a.k.d / 32);
   const long long want = (units + kWarps - 1) / kWarps;
   const int grid = (int)(want < (long long)num_sms * 8 ? want : (long long)num_sms * 8);
-  if (encode)
-    kivi_encode_kernel<G, BITS><<<grid, kWarps * 32, 0, st>>>(a);
-  else
+  if (encode) {
+    auto kern = kivi_encode_kernel<G, BITS>;
+    constexpr int smem = kivi_encode_smem<G>();
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kWarps * 32, smem, st>>>(a);
+  } else {
     kivi_decode_kernel<G, BITS><<<grid, kWarps * 32, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 template <int G>
