@@ -50,6 +50,20 @@ __device__ inline void load_gauge(float* Gs, const CodecArgs& a, long long slice
   __syncwarp();
 }
 
+// The same, transposed per group (Gs[rr][j][i] = G_rr[i][j]), so that one
+// 16-byte load gives four outputs' coefficients of input j.
+template <int G>
+__device__ inline void load_gauge_t(float* Gs, const CodecArgs& a, long long slice, int cg, int lane) {
+  int l, s, b, h;
+  slice_coords(slice, a.k, l, s, b, h);
+  const float* src = a.G + (gauge_set(l, s, h, a.k) * (a.k.d / G) + cg * (32 / G)) * G * G;
+  for (int e = lane; e < 32 * G; e += 32) {
+    const int rr = e / (G * G), i = (e / G) % G, j = e % G;
+    Gs[(rr * G + j) * G + i] = src[e];
+  }
+  __syncwarp();
+}
+
 }  // namespace
 
 // Shared memory of the encoder per warp: its staged gauge (32 G floats) and a
@@ -75,7 +89,7 @@ __global__ void __launch_bounds__(kWarps * 32) kivi_encode_kernel(CodecArgs a) {
     const long long gkey = ku.slice * 64 + ku.cg;
     if (gkey != loaded) {
       __syncwarp();
-      load_gauge<G>(Gs, a, ku.slice, ku.cg, lane);
+      load_gauge_t<G>(Gs, a, ku.slice, ku.cg, lane);
       loaded = gkey;
     }
     int l, s, b, h;
@@ -95,23 +109,23 @@ __global__ void __launch_bounds__(kWarps * 32) kivi_encode_kernel(CodecArgs a) {
         x[8 * v + 6] = bf16lo(w.w); x[8 * v + 7] = bf16hi(w.w);
       }
     }
-    // y = G x per group: fp32 FMA chain over j in index order from +0
+    // y = G x per group: fp32 FMA chain over j in index order from +0, two
+    // outputs' chains per packed fma.rn.f32x2 (each half rounds as the scalar FMA)
     float y[32];
 #pragma unroll
     for (int rr = 0; rr < 32 / G; ++rr) {
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
-        float acc = 0.0f;
-        const float* gi = Gs + (rr * G + i) * G;
+      for (int i = 0; i < G; i += 4) {
+        f2_t acc01 = f2_make(0.0f, 0.0f), acc23 = f2_make(0.0f, 0.0f);
 #pragma unroll
-        for (int j = 0; j < G; j += 4) {
-          const float4 c = *reinterpret_cast<const float4*>(gi + j);
-          acc = __fmaf_rn(c.x, x[rr * G + j + 0], acc);
-          acc = __fmaf_rn(c.y, x[rr * G + j + 1], acc);
-          acc = __fmaf_rn(c.z, x[rr * G + j + 2], acc);
-          acc = __fmaf_rn(c.w, x[rr * G + j + 3], acc);
+        for (int j = 0; j < G; ++j) {
+          const float4 c = *reinterpret_cast<const float4*>(Gs + (rr * G + j) * G + i);
+          const f2_t xx = f2_make(x[rr * G + j], x[rr * G + j]);
+          acc01 = f2_fma(f2_make(c.x, c.y), xx, acc01);
+          acc23 = f2_fma(f2_make(c.z, c.w), xx, acc23);
         }
-        y[rr * G + i] = acc;
+        f2_split(acc01, y[rr * G + i], y[rr * G + i + 1]);
+        f2_split(acc23, y[rr * G + i + 2], y[rr * G + i + 3]);
       }
     }
     if (a.gauged) {
