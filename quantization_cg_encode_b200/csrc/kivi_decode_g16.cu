@@ -18,8 +18,10 @@
 //     (a unit whose |y| could leave the fp16 range is scaled by a power of
 //     two, exactly undone afterwards).
 // The k order of A and B is permuted consistently (each thread reads 4
-// adjacent channels).  The bf16 tile goes through a padded shared-memory
-// staging with stmatrix and leaves with full-line 16-byte stores.
+// adjacent channels).  Each bf16 16-token tile goes through a padded shared-
+// memory staging with stmatrix and leaves with full-line 16-byte stores.  The
+// per-warp buffers are sized by the code width, so that two CTAs (16 warps)
+// share an SM at every code width.
 #include "cg_kernels.cuh"
 
 namespace cg {
@@ -28,12 +30,17 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kPitch = 2 * 128 + 16;  // staging row: 256 B + 16 B pad (distinct bank groups per 8 rows)
-constexpr int kStg = 32 * kPitch;
-constexpr int kCodeBuf = 512 * 8;     // codes of a unit at up to 8 bits
-// per warp: output staging, then two input buffers (codes + 16 B slack, steps,
-// zero points), then the column sums of G
-constexpr int kInBuf = kCodeBuf + 16 + 2 * 256;
-constexpr int kWarpSmem = kStg + 2 * kInBuf + 512;
+constexpr int kStg = 16 * kPitch;     // one 16-token tile
+// per warp: output staging, then two input buffers (the unit's 512 b code
+// bytes + 16 B slack, steps, zero points), then the column sums of G
+template <int BITS>
+__host__ __device__ constexpr int in_buf_bytes() {
+  return 512 * BITS + 16 + 2 * 256;
+}
+template <int BITS>
+__host__ __device__ constexpr int warp_smem_bytes() {
+  return kStg + 2 * in_buf_bytes<BITS>() + 512;
+}
 
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -87,10 +94,11 @@ __device__ __forceinline__ uint32_t bits_at(const unsigned char* p, int bit) {
 }  // namespace
 
 template <int BITS>
-__global__ void __launch_bounds__(kWarps * 32, 1) kivi_decode_g16_kernel(CodecArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 2) kivi_decode_g16_kernel(CodecArgs a) {
   constexpr int D = 128, NG = 8;
   constexpr uint32_t M = (1u << BITS) - 1u;
   constexpr int UNIT_BYTES = 512 * BITS;
+  constexpr int kCodeBuf = UNIT_BYTES, kInBuf = in_buf_bytes<BITS>(), kWarpSmem = warp_smem_bytes<BITS>();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* base = smem_raw + warp * kWarpSmem;
@@ -251,31 +259,33 @@ __global__ void __launch_bounds__(kWarps * 32, 1) kivi_decode_g16_kernel(CodecAr
           }
         }
         // tiles (rows 0-7 | 8-15 of this 16-token tile) x (cols 16r .. +7 | 16r+8 .. +15)
-        stmatrix_x4(st_addr + 16 * tt * kPitch + 32 * r, pk[0][0], pk[0][1], pk[1][0], pk[1][1]);
+        stmatrix_x4(st_addr + 32 * r, pk[0][0], pk[0][1], pk[1][0], pk[1][1]);
       }
-    }
-    __syncwarp();
-    // 32 rows of 256 B, contiguous in the output: each instruction writes two whole rows
-    uint16_t* obase = a.kv_out + (slice * a.k.T + 32LL * tgroup) * D;
+      __syncwarp();
+      // the tile's 16 rows of 256 B, contiguous in the output: each instruction writes two whole rows
+      uint16_t* obase = a.kv_out + (slice * a.k.T + 32LL * tgroup + 16 * tt) * D;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int row = 2 * k + (lane >> 4), ch = lane & 15;
-      reinterpret_cast<uint4*>(obase + row * D)[ch] = *reinterpret_cast<const uint4*>(stg + row * kPitch + ch * 16);
+      for (int k = 0; k < 8; ++k) {
+        const int row = 2 * k + (lane >> 4), ch = lane & 15;
+        reinterpret_cast<uint4*>(obase + row * D)[ch] = *reinterpret_cast<const uint4*>(stg + row * kPitch + ch * 16);
+      }
+      __syncwarp();
     }
-    __syncwarp();
   }
 }
 
 namespace {
-constexpr int kSmem = kWarps * kWarpSmem;
 template <int BITS>
 cudaError_t kd_launch(const CodecArgs& a, int num_sms, cudaStream_t st) {
+  constexpr int kSmem = kWarps * warp_smem_bytes<BITS>();
+  // CTAs per SM: two where their shared memory (plus 1 KB reserved per CTA) fits in 228 KB (every width)
+  constexpr int kCtas = 2 * (kSmem + 1024) <= 228 * 1024 ? 2 : 1;
   auto kern = kivi_decode_g16_kernel<BITS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   const long long units = a.k.slices() * (a.nt / 32);
   const long long want = (units + kWarps - 1) / kWarps;
-  const int grid = (int)(want < num_sms ? want : num_sms);
+  const int grid = (int)(want < (long long)num_sms * kCtas ? want : (long long)num_sms * kCtas);
   kern<<<grid, kWarps * 32, kSmem, st>>>(a);
   return cudaGetLastError();
 }
