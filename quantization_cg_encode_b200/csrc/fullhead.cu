@@ -8,15 +8,16 @@
 //
 // Encode, per block of 128 tokens of one head slice:
 //   * a TMA warp streams x blocks (128 x 128 bf16 = 32 KB, two 16 KB boxes with
-//     128-byte swizzle, no multicast) into a 3-stage shared-memory ring, and
+//     128-byte swizzle, no multicast) into a 4-stage shared-memory ring, and
 //     writes each head slice's G as bf16 (RNE) in the same swizzled K-major
 //     layout (two buffers, so the next slice's G is staged while the current
 //     one is in use);
 //   * one thread issues 8 tcgen05.mma (M = N = 128, K = 16, bf16 x bf16 -> fp32)
-//     into one of two 128-column TMEM accumulators: y[t][i] = sum_j x[t][j] G[i][j];
-//   * four epilogue warps (one thread per token) read their row with
-//     tcgen05.ld, reduce the 16-token ranges with half-warp shuffles and
-//     quantize, pack and store exactly like the grouped encoder.
+//     into one of four 128-column TMEM accumulators: y[t][i] = sum_j x[t][j] G[i][j];
+//   * three epilogue warpgroups take blocks in turn (one thread per token):
+//     a first pass over the row's TMEM columns gives its range, half-warp
+//     shuffles the 16-token block's; a second pass quantizes, packs and
+//     stores the codes 32 at a time, as the grouped encoder defines them.
 // Every wait on an mbarrier is bounded in time.
 #include <cuda.h>
 
@@ -335,13 +336,14 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
   }
 }
 
-
 // Decode, per block of 128 tokens: x_hat_t = G^T (s q_t + z) = s (G^T q_t) + z (G^T 1)
-// (the range block of 16 tokens x d_head has one s and z).  Four warps expand
-// the codes into the A operand (exact bf16 integers, swizzled K-major rows in
-// shared memory) for block i+1 while the tensor cores contract block i with
+// (the range block of 16 tokens x d_head has one s and z).  Two warpgroups take
+// alternate blocks, each with its own A buffer and accumulator: a warpgroup
+// expands its block's codes into the A operand (exact bf16 integers, swizzled
+// K-major rows in shared memory), the tensor cores contract it with
 // B = G^T (bf16, swizzled K-major, column sums of the same bf16 values kept
-// beside it); the same warps then read the accumulator and write bf16.
+// beside it), and the same warps then read the accumulator and write bf16,
+// while the other warpgroup works on the next block.
 namespace {
 constexpr int kDecEpi = 8;  // two warpgroups taking alternate blocks: code expansion, then epilogue
 constexpr int kDecThreads = (kDecEpi + 2) * 32;

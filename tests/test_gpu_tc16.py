@@ -81,7 +81,8 @@ def test_ragged_token_ranges(t0, nt):
 
 def test_many_blocks_per_cta_and_slice_changes():
     """512 blocks of 128 tokens over 148 SMs: each CTA crosses head slices (G restaged,
-    both TMEM buffers of both epilogue warpgroups reused), with a ragged tail per slice."""
+    its four TMEM accumulators reused by the three epilogue warpgroups), with a ragged
+    tail per slice."""
     need_gpu()
     kv = synth.kv_cache(2, 1, 4, 4096, 128, seed=11, device="cuda", n_outliers=4)
     _, _, _, ref, y = _check(kv, _oracle_G(2, 4, seed=11), 4, 0, 4096 - 48)
