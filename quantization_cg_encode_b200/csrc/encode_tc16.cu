@@ -656,7 +656,7 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
       }
     }
   } else {
-    // ---------------- epilogue: two warpgroups, thread = token row ----------------
+    // ---------------- epilogue: three warpgroups, thread = token row ----------------
     const int wg = (warp - 2) >> 2;
     const int quarter = warp & 3;  // TMEM lanes this warp may read
     const int row = 32 * quarter + lane;
