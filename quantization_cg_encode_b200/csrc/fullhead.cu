@@ -343,7 +343,9 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
 // K-major rows in shared memory), the tensor cores contract it with
 // B = G^T (bf16, swizzled K-major, column sums of the same bf16 values kept
 // beside it), and the same warps then read the accumulator and write bf16,
-// while the other warpgroup works on the next block.
+// while the other warpgroup works on the next block.  A warpgroup's loads of
+// its next block's codes are issued as soon as the current block's are
+// expanded, so they are in flight during its epilogue.
 namespace {
 constexpr int kDecEpi = 8;  // two warpgroups taking alternate blocks: code expansion, then epilogue
 constexpr int kDecThreads = (kDecEpi + 2) * 32;
@@ -497,9 +499,30 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
     // thread = token row (the other warpgroup's work covers this block's MMA) ----------------
     const int wg = warp >> 2, quarter = warp & 3;
     const int row = 32 * quarter + lane;
+    // this thread's codes of block (sl, q): its token row's 16 BITS bytes (rows past
+    // the range repeat a valid row)
+    auto load_codes = [&](long long sl, int q, uint4 (&dst)[BITS]) {
+      const int valid = min(128, a.nt - 128 * q);
+      const int tok = a.t0 + 128 * q + min(row, valid - 1);
+      const uint4* src = reinterpret_cast<const uint4*>(a.codes_in + sl * slice_code_bytes +
+                                                        (long long)(tok / 16) * (16 * D * BITS / 8) +
+                                                        (tok % 16) * (D * BITS / 8));
+#pragma unroll
+      for (int w = 0; w < BITS; ++w) dst[w] = __ldg(src + w);
+    };
     long long slice = b0 / bps;
     int bq = (int)(b0 - slice * bps);
     int gcount = 0;
+    uint4 next[BITS];  // codes of this warpgroup's next block, loading while it finishes the current one
+    if (wg < n_blocks) {
+      long long sl = slice;
+      int q = bq + wg;
+      if (q >= bps) {
+        q -= bps;
+        ++sl;
+      }
+      load_codes(sl, q, next);
+    }
     for (int i = 0; i < n_blocks; ++i) {
       const int gb = gcount & 1;
       const bool last_of_slice = (bq + 1 == bps) || (i + 1 == n_blocks);
@@ -507,18 +530,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
         const int ab = i & 1;  // == wg: each warpgroup has its own A buffer and accumulator
         const int valid = min(128, a.nt - 128 * bq);
         {  // codes of the block -> exact bf16 integers, swizzled K-major A operand
-          mbar_wait(&sm.a_empty[ab], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.status);
-          const int tok = a.t0 + 128 * bq + min(row, valid - 1);  // rows past the range repeat a valid row
-          const uint4* src = reinterpret_cast<const uint4*>(a.codes_in + slice * slice_code_bytes +
-                                                            (long long)(tok / 16) * (16 * D * BITS / 8) +
-                                                            (tok % 16) * (D * BITS / 8));
           uint32_t words[4 * BITS + 1];
 #pragma unroll
           for (int w = 0; w < BITS; ++w) {
-            const uint4 v = src[w];
+            const uint4 v = next[w];
             words[4 * w] = v.x; words[4 * w + 1] = v.y; words[4 * w + 2] = v.z; words[4 * w + 3] = v.w;
           }
           words[4 * BITS] = 0;
+          if (i + 2 < n_blocks) {  // block i + 2 is this warpgroup's next
+            long long sl = slice;
+            int q = bq + 2;
+            while (q >= bps) {  // at most twice
+              q -= bps;
+              ++sl;
+            }
+            load_codes(sl, q, next);
+          }
+          mbar_wait(&sm.a_empty[ab], ((uint32_t)(i >> 1) & 1u) ^ 1u, a.status);
           unsigned char* adst = sm.as + ab * kBlockBytes;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {  // 16-byte chunk c = channels 8c .. 8c+7
