@@ -7,7 +7,8 @@ bit settings (2, 3, 4, 6, 8 bits/value; 3, 4, 6 in the main results).  The
 pages print no quantizer formula.  This module takes the plainest asymmetric
 min/max reading, with every floating-point step an IEEE fp32 operation in RNE:
 
-  mn, mx = min(y), max(y) over the range block            (exact)
+  mn, mx = min(y), max(y) over the range block            (exact; a zero
+                                                            extreme is +0)
   z      = fp16_rne(clamp(mn, +-65504))                     zero point (offset)
   s      = fp16_rne(min(fl32(fl32(mx - mn) / (2^b - 1)), 65504))   step
   s == 0 -> every code is 0
@@ -25,10 +26,16 @@ from .fpround import fl16, fl32, F16_MAX
 
 
 def quant_params(mn, mx, bits):
-    """fp16 zero point z and step s of a range block, returned as float64."""
+    """fp16 zero point z and step s of a range block, returned as float64.
+
+    The range ends are real numbers: -0 and +0 are the same value, so a zero
+    minimum or maximum is taken as +0 (adding +0 maps -0 to +0 and leaves
+    every other value unchanged), and the stored zero point of a block whose
+    minimum is zero is the fp16 +0.
+    """
     qmax = float(2 ** bits - 1)
-    mn = np.asarray(mn, dtype=np.float64)
-    mx = np.asarray(mx, dtype=np.float64)
+    mn = np.asarray(mn, dtype=np.float64) + 0.0
+    mx = np.asarray(mx, dtype=np.float64) + 0.0
     z = fl16(np.clip(mn, -F16_MAX, F16_MAX))
     rng = fl32(mx - mn)
     s32 = fl32(rng / qmax)

@@ -138,3 +138,16 @@ def test_kivi_sizes_and_round_trip_error():
     xr = oc.decode_kivi(enc, G32, 3)
     rel = np.sqrt(((xr - x) ** 2).sum() / (x ** 2).sum())
     assert 0.01 < rel < 0.2
+
+
+def test_zero_extremes_are_positive_zero():
+    """-0 and +0 are one real number: a block whose minimum (or whole range) is
+    zero stores the fp16 +0 as its zero point and step, whichever zero the
+    values carry and in whatever order they come."""
+    for blk in ([-0.0, 0.0, 1.0], [0.0, -0.0, 1.0], [-0.0, 2.0], [-0.0, -0.0], [0.0, -0.0]):
+        q, z, s = oq.quantize_ranges(np.array([blk]), 4)
+        assert np.signbit(z).sum() == 0 and np.signbit(s).sum() == 0, blk
+        assert np.asarray(z, np.float16).view(np.uint16)[0] == 0
+    # a negative minimum keeps its sign, and a non-zero block is unchanged
+    q, z, s = oq.quantize_ranges(np.array([[-0.5, 1.0]]), 4)
+    assert z[0] == -0.5 and s[0] == fl16(fl32(1.5 / 15))
