@@ -58,12 +58,28 @@ typedef enum {
   CG_QUANT_KIVI = 1           /* keys per channel, values per token           */
 } cg_quant_mode;
 
-/* Where the gauge contraction of cg_encode runs.  Codes, steps and zero points
- * do not depend on it; only the optional gauged output does. */
+/* Which gauge contraction feeds the quantizer in cg_encode.  The codes, steps
+ * and zero points are always the quantizer's exact fp32 result for the gauged
+ * values that engine produced (returned through the optional gauged output);
+ * the engines differ in how those gauged values are defined.  Decode does not
+ * depend on the engine. */
 typedef enum {
-  CG_ENGINE_AUTO = 0,      /* tensor cores where a kernel exists (g = 16 with
-                              d = 128 and W = g, and g = d), else CUDA cores */
-  CG_ENGINE_CUDA_CORES = 1 /* the fp32 FMA chain on CUDA cores (g < d only)  */
+  CG_ENGINE_AUTO = 0,         /* the fastest kernel for the request:
+                                 g = 16 with W = 16 (d 64 or 128): tensor-core
+                                 contraction with G split into two bf16 terms
+                                 (within about 2^-17 sum_j |G_ij x_j| of G x);
+                                 g = d: tensor cores with G rounded to bf16;
+                                 otherwise the fp32 FMA chain */
+  CG_ENGINE_CUDA_CORES = 1,   /* the fp32 FMA chain on CUDA cores (g < d only):
+                                 y_i = fl32(G_ij x_j + acc), j = 0..g-1 from +0,
+                                 bit-reproducible on any device */
+  CG_ENGINE_CHAIN_TENSOR = 2  /* the same codes as CG_ENGINE_CUDA_CORES, with the
+                                 contraction on the 5th-generation tensor cores
+                                 (g = 16, d = 128, W = 16 only): G split exactly
+                                 into three bf16 terms, and the chain re-evaluated
+                                 wherever the tensor-core value could change a
+                                 decision (needs G orthogonal to 2^-12, checked
+                                 per head slice; else the chain throughout) */
 } cg_engine;
 
 /* Shape of a KV cache: K_l, V_l in R^{B x H x T x d} for l = 1..L
@@ -86,7 +102,7 @@ typedef struct {
  *               (the page's "one range per T_b x d_l block").
  *   mode        cg_quant_mode.
  *   kivi_key_tokens, kivi_val_channels: KIVI group sizes, both 32.
- *   engine      cg_engine (encode only).
+ *   engine      cg_engine (encode only; decode ignores it).
  */
 typedef struct {
   int32_t g;
@@ -157,17 +173,13 @@ cg_status cg_gauge_build(const float* A_dev, float* G_dev, int32_t n_mats, int32
  * zeros [..][T/32][d] and [..][T][d/32].
  * Per range: z = fp16(min), s = fp16(fl32(fl32(max - min) / (2^b - 1))),
  * q = clamp(rne(fl32(fl32(y - z) * fl32(1/s))), 0, 2^b - 1), q = 0 if s = 0.
- * Gauged values: for g < d each y_i is the fp32 fused-multiply-add chain over
- * j = 0..g-1 in index order (bit-reproducible); for g = d the contraction runs
- * on the tensor cores with G rounded to bf16 and fp32 accumulation.
- * For g < d the codes, steps and zero points are those of the chain whatever
- * the engine: the tensor-core encoder (g = 16, d = 128, W = g) contracts with
- * G split exactly into three bf16 terms and re-evaluates the chain wherever
- * the tensor-core value could change a decision, which relies on G having
- * orthonormal rows (checked per head slice; a gauge that is not orthogonal to
- * 2^-12 is evaluated with the chain throughout).  Its gauged output then
- * holds the values it quantized: within 2^-16 max|y| of the block (16 x 16)
- * of the chain, and equal to it wherever the chain was evaluated. */
+ * Gauged values: see cg_engine.  Whatever the engine, the codes, steps and
+ * zero points equal the quantizer above applied to the gauged values the
+ * engine produced (bit for bit), and a zero block minimum or maximum is taken
+ * as +0.  With CG_ENGINE_CHAIN_TENSOR the gauged output holds the values
+ * actually quantized: within 2^-16 max|y| of the 16 x 16 block of the chain
+ * and equal to it wherever the chain was evaluated, while the codes are the
+ * chain's. */
 cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec,
                     const void* kv_dev, const float* G_dev, int32_t t0, int32_t nt,
                     uint8_t* codes_dev, void* scales_dev, void* zeros_dev,

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libcg.so")
 
 CG_OK, CG_ERR_INVALID, CG_ERR_UNSUPPORTED, CG_ERR_CUDA, CG_ERR_TIMEOUT, CG_ERR_TOO_LARGE = range(6)
 BLOCK_UNIFORM, KIVI = 0, 1
-ENGINE_AUTO, ENGINE_CUDA_CORES = 0, 1
+ENGINE_AUTO, ENGINE_CUDA_CORES, ENGINE_CHAIN_TENSOR = 0, 1, 2
 
 # Every symbol include/cg.h declares.
 EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",

@@ -42,8 +42,12 @@ cg_status check_codec(const cg_kv_desc* kv, const cg_codec_desc* c) {
   } else {
     return CG_ERR_INVALID;
   }
-  if (c->engine != CG_ENGINE_AUTO && c->engine != CG_ENGINE_CUDA_CORES) return CG_ERR_INVALID;
+  if (c->engine != CG_ENGINE_AUTO && c->engine != CG_ENGINE_CUDA_CORES && c->engine != CG_ENGINE_CHAIN_TENSOR)
+    return CG_ERR_INVALID;
   if (c->engine == CG_ENGINE_CUDA_CORES && c->g == d) return CG_ERR_UNSUPPORTED;
+  if (c->engine == CG_ENGINE_CHAIN_TENSOR &&
+      !(c->g == 16 && d == 128 && c->mode == CG_QUANT_BLOCK_UNIFORM && c->range_cols == 16))
+    return CG_ERR_UNSUPPORTED;
   return CG_OK;
 }
 
@@ -159,8 +163,9 @@ cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec, const void
     if (kv->d_head != 128) return CG_ERR_UNSUPPORTED;
     return from_cuda(launch_fullhead(a, true, num_sms(), (cudaStream_t)stream));
   }
-  if (codec->engine == CG_ENGINE_AUTO && encode_tc16_supported(a))
-    return from_cuda(launch_encode_tc16(a, num_sms(), (cudaStream_t)stream));
+  if (codec->engine == CG_ENGINE_CHAIN_TENSOR) return from_cuda(launch_encode_tc16(a, num_sms(), (cudaStream_t)stream));
+  if (codec->engine == CG_ENGINE_AUTO && codec_mma16_supported(a))
+    return from_cuda(launch_encode_mma16(a, num_sms(), (cudaStream_t)stream));
   if (a.g == 16) return from_cuda(launch_encode_g16(a, num_sms(), (cudaStream_t)stream));
   return from_cuda(launch_group_codec(a, true, num_sms(), (cudaStream_t)stream));
 }
@@ -198,6 +203,7 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec, const uint
     if (kv->d_head != 128) return CG_ERR_UNSUPPORTED;
     return from_cuda(launch_fullhead(a, false, num_sms(), (cudaStream_t)stream));
   }
+  if (codec_mma16_supported(a)) return from_cuda(launch_decode_mma16(a, num_sms(), (cudaStream_t)stream));
   if (a.g == 16) return from_cuda(launch_decode_g16(a, num_sms(), (cudaStream_t)stream));
   return from_cuda(launch_group_codec(a, false, num_sms(), (cudaStream_t)stream));
 }

@@ -90,7 +90,8 @@ __device__ __forceinline__ float warp_max_f32(float v) {
 }
 
 // ---- the quantizer's block parameters -------------------------------------------------
-// z = fp16_rne(clamp(mn)), s = fp16_rne(min(fl32(fl32(mx - mn) / qmax), 65504)).
+// z = fp16_rne(clamp(mn)), s = fp16_rne(min(fl32(fl32(mx - mn) / qmax), 65504)),
+// with a zero minimum or maximum taken as +0.
 // The division by the integer qmax = 2^b - 1 is evaluated as the fp64 product
 // r * fl64(1/qmax) rounded to fp32, which equals the correctly rounded fp32
 // quotient Q = r / qmax: (i) Q is never an fp32 rounding midpoint, because a
@@ -107,6 +108,8 @@ struct QParams {
 
 __device__ __forceinline__ QParams quant_params(float mn, float mx, double inv_qmax) {
   QParams p;
+  mn = __fadd_rn(mn, 0.0f);  // a zero extreme is +0 (-0 + +0 = +0)
+  mx = __fadd_rn(mx, 0.0f);
   float zc = fminf(fmaxf(mn, -65504.0f), 65504.0f);
   __half z = __float2half_rn(zc);
   float rng = __fsub_rn(mx, mn);
@@ -153,25 +156,25 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Wait for phase `parity` of `bar` to complete.  Gives up after kWaitNs of
 // wall time, ORs kStatusTimeout into *status and returns false (the caller
 // carries on, so every thread still reaches every barrier and the kernel ends).
+__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return done;
+}
+// (The first test needs no clock: the common case is a phase already complete.)
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status) {
   const uint32_t addr = smem_u32(bar);
-  uint64_t t0 = 0;
-  for (uint32_t i = 0;; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if ((i & 255u) == 0) {
-      const uint64_t now = global_ns();
-      if (i == 0) {
-        t0 = now;
-      } else if (now - t0 > kWaitNs) {
-        atomicOr(status, kStatusTimeout);
-        return false;
-      }
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if ((i & 255u) == 0 && global_ns() - t0 > kWaitNs) {
+      atomicOr(status, kStatusTimeout);
+      return false;
     }
   }
 }

@@ -182,6 +182,7 @@ __device__ __forceinline__ void stats16(const float* y, float& mn, float& mx, fl
 // fp16 bits of the zero point and step the quantizer would derive from a range
 // end / width (the same operations as quant_params, monotone in the argument).
 __device__ __forceinline__ uint16_t z_bits(float mn) {
+  mn = __fadd_rn(mn, 0.0f);  // a zero minimum is +0
   return __half_as_ushort(__float2half_rn(fminf(fmaxf(mn, -65504.0f), 65504.0f)));
 }
 // The step from a range width: fp16(min(fl32(rng / qmax), 65504)).  The fp32

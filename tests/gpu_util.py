@@ -41,10 +41,44 @@ def run_decode(kv_shape, G, codec, codes, scales, zeros, t0=0, nt=None, fill=0.0
     return out
 
 
-def tensor_core_g16(shape, codec):
-    """True when cg_encode runs the tensor-core g = 16 encoder for this request."""
-    return (codec.g == 16 and shape[-1] == 128 and codec.range_cols == 16 and codec.mode == cg.BLOCK_UNIFORM
+def chain_tensor_g16(shape, codec):
+    """True when cg_encode runs the chain-exact tensor-core g = 16 encoder."""
+    return codec.engine == cg.ENGINE_CHAIN_TENSOR
+
+
+def own_gauge_g16(shape, codec):
+    """True when cg_encode's gauged values are its own two-term tensor-core
+    contraction (the default engine for g = 16 with 16 x 16 ranges)."""
+    return (codec.g == 16 and shape[-1] in (64, 128) and codec.range_cols == 16 and codec.mode == cg.BLOCK_UNIFORM
             and codec.engine == cg.ENGINE_AUTO)
+
+
+def oracle_quantize_own(y, bits, w):
+    """The oracle's block-uniform quantizer applied to the device's fp32 gauged
+    values y [..., T, d]: dict(codes, z, s, q) in the oracle's layout."""
+    from oracle import quant as oq
+    q, z, s = oq.quantize_ranges(oq.block_uniform_view(np.asarray(y, np.float64), 16, w), bits)
+    return dict(codes=oq.pack_codes(q, bits), z=z, s=s, q=q)
+
+
+OWN_GAUGE_BOUND = 2.0 ** -16
+
+
+def assert_gauge_within(y_dev, x, G, bound=OWN_GAUGE_BOUND, what=""):
+    """|y_dev - G x| <= bound * sum_j |G_ij x_j| for every value (G x exact, fp64),
+    and the per-slice norm-relative error far inside 2e-3."""
+    from oracle import gauge as og
+    y_dev = np.asarray(y_dev, np.float64)
+    ref = og.apply_gauge(x, G)
+    mag = og.apply_gauge(np.abs(x), np.abs(np.asarray(G, np.float64)))
+    err = np.abs(y_dev - ref)
+    bad = err > bound * mag
+    assert not bad.any(), "%s: %d gauged values beyond %.3g sum|G x|, worst ratio %.3g" % (
+        what, int(bad.sum()), bound, float((err / np.maximum(mag, 1e-300)).max()))
+    flat_e = (y_dev - ref).reshape(-1, ref.shape[-2] * ref.shape[-1])
+    flat_r = ref.reshape(flat_e.shape)
+    rel = np.sqrt((flat_e ** 2).sum(-1)) / np.maximum(np.sqrt((flat_r ** 2).sum(-1)), 1e-300)
+    assert rel.max() <= 2e-3, "%s: slice norm-relative error %.3g" % (what, rel.max())
 
 
 def block_uniform_np(codes, scales, zeros, shape, codec):

@@ -76,7 +76,11 @@ def test_encode_validation_without_gpu():
     assert _enc(cg.kv_desc(1, 1, 2, 1024, 96), cg.codec_desc(g=16, bits=4), nt=0) == cg.CG_ERR_UNSUPPORTED
     kivi = cg.codec_desc(g=16, bits=3, mode=cg.KIVI)
     assert _enc(kvd, kivi, t0=16, nt=32) == cg.CG_ERR_INVALID              # KIVI needs 32-token steps
-    assert _enc(kvd, cg.codec_desc(g=16, bits=4, engine=2), nt=16) == cg.CG_ERR_INVALID   # unknown engine
+    assert _enc(kvd, cg.codec_desc(g=16, bits=4, engine=7), nt=16) == cg.CG_ERR_INVALID   # unknown engine
+    chain_tc = cg.codec_desc(g=16, bits=4, engine=cg.ENGINE_CHAIN_TENSOR)
+    assert _enc(cg.kv_desc(1, 1, 2, 1024, 64), chain_tc, nt=16) == cg.CG_ERR_UNSUPPORTED  # d = 128 only
+    chain_w = cg.codec_desc(g=16, bits=4, range_cols=128, engine=cg.ENGINE_CHAIN_TENSOR)
+    assert _enc(cg.kv_desc(1, 1, 2, 1024, 128), chain_w, nt=16) == cg.CG_ERR_UNSUPPORTED  # 16 x 16 ranges only
     full = cg.codec_desc(g=128, bits=4, range_cols=128, engine=cg.ENGINE_CUDA_CORES)
     assert _enc(cg.kv_desc(1, 1, 2, 1024, 128), full, nt=16) == cg.CG_ERR_UNSUPPORTED  # full head: tensor cores only
 

@@ -1,9 +1,12 @@
 """GPU parity of the grouped-gauge block-uniform codec against the oracle.
 
-Codes, scales and zero points must match the oracle bit for bit; the gauged
-values the quantizer saw (the fp32 FMA chain) must match bit for bit; decoded
-reconstructions must match the oracle's fp64 G^T (s q + z) within the bf16
-tolerance (per-slice norm-relative 2e-3 plus an elementwise half-ulp bound).
+Codes, scales and zero points must match the oracle's quantizer bit for bit,
+given the gauged values the kernel quantized: the fp32 FMA chain (g = 8, 32,
+16 x d ranges, the CUDA-core engine), which must itself match the oracle's
+chain bit for bit, or the default g = 16 engine's own two-term tensor-core
+contraction, which must lie within 2^-16 sum_j |G_ij x_j| of the exact G x.
+Decoded reconstructions must match the oracle's fp64 G^T (s q + z) within the
+bf16 tolerance (per-slice norm-relative 2e-3 plus an elementwise half-ulp bound).
 """
 import numpy as np
 import pytest
@@ -13,8 +16,8 @@ from oracle import codec as oc
 from oracle import gauge as og
 from oracle import quant as oq
 from quantization_cg_encode_b200 import cg, synth
-from tests.gpu_util import (assert_close_bf16, bf16_np, block_uniform_np, need_gpu, run_decode, run_encode,
-                            tensor_core_g16)
+from tests.gpu_util import (assert_close_bf16, assert_gauge_within, bf16_np, block_uniform_np, chain_tensor_g16,
+                            need_gpu, oracle_quantize_own, own_gauge_g16, run_decode, run_encode)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,23 +34,33 @@ def _inputs(L, B, H, T, d, g, seed=0, sigma=0.1, n_outliers=None, outliers=(3, 1
 
 
 def _check_encode(kv, G, codec, t0=0, nt=None):
+    """Encode on the GPU and check it against the oracle.  Chain engines: codes,
+    steps, zero points and gauged values equal the oracle's fp32 chain.  The
+    default g = 16 engine: codes, steps and zero points equal the oracle's
+    quantizer applied to the kernel's own gauged values, which lie within the
+    two-term tensor-core bound of the exact G x.  Returns the reference codes
+    (equal to the device's) for the decode check."""
     T = kv.shape[4]
     nt = T - t0 if nt is None else nt
     codes, scales, zeros, gauged = run_encode(kv, G, codec, t0, nt)
     x = bf16_np(kv)
     G32 = G.cpu().numpy().astype(np.float64)
-    ref = oc.encode_block_uniform(x, G32, codec.bits, tb=16, w=codec.range_cols, t0=t0, nt=nt)
     c, s, z = block_uniform_np(codes, scales, zeros, kv.shape, codec)
     tb0, tb1 = t0 // 16, (t0 + nt) // 16
     y = gauged.cpu().numpy().astype(np.float64)
-    if tensor_core_g16(kv.shape, codec):
-        # the tensor-core encoder reports the values it quantized: within 2^-16 of the
-        # block maximum from the chain (its codes are the chain's, checked below)
-        d = oq.block_uniform_view(np.abs(y[..., t0:t0 + nt, :] - ref["y"]), 16, 16).max(-1)
-        m = oq.block_uniform_view(np.abs(ref["y"]), 16, 16).max(-1)
-        assert np.all(d <= 2.0 ** -16 * m), "gauged values beyond the tensor-core bound"
+    if own_gauge_g16(kv.shape, codec):
+        assert_gauge_within(y[..., t0:t0 + nt, :], x[..., t0:t0 + nt, :], G32, what="gauged values")
+        ref = oracle_quantize_own(y[..., t0:t0 + nt, :], codec.bits, codec.range_cols)
     else:
-        assert np.array_equal(y[..., t0:t0 + nt, :], ref["y"]), "gauged values differ from the fp32 chain"
+        ref = oc.encode_block_uniform(x, G32, codec.bits, tb=16, w=codec.range_cols, t0=t0, nt=nt)
+        if chain_tensor_g16(kv.shape, codec):
+            # the chain-exact tensor-core encoder reports the values it quantized: within
+            # 2^-16 of the block maximum from the chain (its codes are the chain's)
+            d = oq.block_uniform_view(np.abs(y[..., t0:t0 + nt, :] - ref["y"]), 16, 16).max(-1)
+            m = oq.block_uniform_view(np.abs(ref["y"]), 16, 16).max(-1)
+            assert np.all(d <= 2.0 ** -16 * m), "gauged values beyond the tensor-core bound"
+        else:
+            assert np.array_equal(y[..., t0:t0 + nt, :], ref["y"]), "gauged values differ from the fp32 chain"
     assert np.all(np.isnan(y[..., :t0, :])) and np.all(np.isnan(y[..., t0 + nt:, :])), "wrote outside the range"
     assert np.array_equal(z[..., tb0:tb1, :], np.asarray(ref["z"]).astype(np.float16).view(np.uint16))
     assert np.array_equal(s[..., tb0:tb1, :], np.asarray(ref["s"]).astype(np.float16).view(np.uint16))
@@ -133,13 +146,19 @@ def test_gauge_build_group_and_full_head():
 @pytest.mark.parametrize("bits", [3, 4, 6])
 def test_8b_shaped_cache_sampled_parity(bits):
     """Full 8B-shaped cache (32 x 2 x 8 x 4096 x 128) in the launch configuration the
-    benchmark times; the oracle checks sampled (l, s, h) slices exactly."""
+    benchmark times (no gauged output): its codes equal those of a second run that
+    also writes the gauged values, and on sampled (l, s, h) slices the oracle checks
+    them (its quantizer on those gauged values), the gauged values themselves and the
+    decode."""
     need_gpu()
     L, B, H, T, d = 32, 1, 8, 4096, 128
     kv = synth.kv_cache(L, B, H, T, d, seed=1, device="cuda", n_outliers=4)
     G = oracle_gauge(synth.gauge_params(L, H, d // 16, 16, sigma=0.1, seed=1))
     codec = cg.codec_desc(g=16, bits=bits)
     codes, scales, zeros, _ = run_encode(kv, G, codec, want_gauged=False)
+    codes2, scales2, zeros2, gauged = run_encode(kv, G, codec, want_gauged=True)
+    assert torch.equal(codes, codes2) and torch.equal(scales, scales2) and torch.equal(zeros, zeros2)
+    del codes2, scales2, zeros2
     out = run_decode(kv.shape, G, codec, codes, scales, zeros)
     c, s, z = block_uniform_np(codes, scales, zeros, kv.shape, codec)
     rng = np.random.default_rng(bits)
@@ -147,7 +166,9 @@ def test_8b_shaped_cache_sampled_parity(bits):
         l, sk, h = int(rng.integers(L)), int(rng.integers(2)), int(rng.integers(H))
         x = bf16_np(kv[l:l + 1, sk:sk + 1, :, h:h + 1])
         Gs = G[l:l + 1, sk:sk + 1, h:h + 1].cpu().numpy().astype(np.float64)
-        ref = oc.encode_block_uniform(x, Gs, bits)
+        y = gauged[l:l + 1, sk:sk + 1, :, h:h + 1].cpu().numpy().astype(np.float64)
+        assert_gauge_within(y, x, Gs, what="8B slice gauged values")
+        ref = oracle_quantize_own(y, bits, 16)
         assert np.array_equal(c[l, sk, :, h], ref["codes"][0, 0, :, 0])
         assert np.array_equal(s[l, sk, :, h], ref["s"][0, 0, :, 0].astype(np.float16).view(np.uint16))
         assert np.array_equal(z[l, sk, :, h], ref["z"][0, 0, :, 0].astype(np.float16).view(np.uint16))

@@ -1,4 +1,5 @@
-"""GPU parity of the tensor-core g = 16 encoder (d_head = 128, 16 x 16 ranges).
+"""GPU parity of the chain-exact tensor-core g = 16 encoder (engine
+CG_ENGINE_CHAIN_TENSOR; d_head = 128, 16 x 16 ranges).
 
 The tensor cores contract with G split exactly into three bf16 terms, and the
 encoder re-evaluates the fp32 FMA chain wherever the tensor-core value could
@@ -26,7 +27,7 @@ def _oracle_G(L, H, sigma=0.1, seed=0):
     return og.gauge_from_A(A.numpy().astype(np.float64)).astype(np.float32)
 
 
-def _check(kv, G32, bits, t0=0, nt=None, engine=cg.ENGINE_AUTO):
+def _check(kv, G32, bits, t0=0, nt=None, engine=cg.ENGINE_CHAIN_TENSOR):
     """Encode on the GPU and compare with the oracle; returns (codes, scales, zeros, ref, y_gpu)."""
     T = kv.shape[4]
     nt = T - t0 if nt is None else nt
