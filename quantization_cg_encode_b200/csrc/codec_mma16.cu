@@ -55,6 +55,22 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// d = a b (no accumulator input: C is a zero register, d is written only, so no
+// zeroing of d is needed before the first product of a chain)
+__device__ __forceinline__ void mma_bf16_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+__device__ __forceinline__ void mma_f16_16816_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -301,9 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
         ldmatrix_x4(afr, xs_lane + s * C::XBYTES + j * 2048);
 #pragma unroll
         for (int nh = 0; nh < 2; ++nh) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[j][nh][e] = 0.0f;
-          mma_bf16_16816(acc[j][nh], afr, bl[nh][0], bl[nh][1]);
+          mma_bf16_16816_z(acc[j][nh], afr, bl[nh][0], bl[nh][1]);
           mma_bf16_16816(acc[j][nh], afr, bh[nh][0], bh[nh][1]);
         }
       }
@@ -580,8 +594,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma16_kernel(CodecArgs a) 
       uint32_t pk[2][2];  // [row g / g+8][channels 4c,4c+1 / 4c+2,4c+3] bf16 pairs
 #pragma unroll
       for (int nh = 0; nh < 2; ++nh) {
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        mma_f16_16816(acc, afr, bl[nh][0], bl[nh][1]);
+        float acc[4];
+        mma_f16_16816_z(acc, afr, bl[nh][0], bl[nh][1]);
         mma_f16_16816(acc, afr, bh[nh][0], bh[nh][1]);
         const float cz0 = zf[j] * csum[2 * nh], cz1 = zf[j] * csum[2 * nh + 1];
         pk[0][nh] = pack_bf16x2(__fmaf_rn(sf[j], acc[0], cz0), __fmaf_rn(sf[j], acc[1], cz1));
