@@ -214,8 +214,10 @@ cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* 
  *   totals_dev   fp64 [4]: sum L_freq, sum L_rate, n_blocks, L  (output)
  *   dG_dev       fp32 [L][2][H][d/g][g][g] = dL/dG, or NULL; requires G_dev
  *   workspace_dev / workspace_bytes: at least cg_spectral_workspace_size().
- * Reductions run in a fixed order: results are deterministic for a given
- * shape. */
+ * Shapes: d_head 64 or 128, T a multiple of 32 (tb = 16, g = 16 or no gauge);
+ * d_head = 128 with T a multiple of 128 runs on the tensor cores, every other
+ * shape on CUDA cores.  Reductions run in a fixed order: results are
+ * deterministic for a given shape. */
 cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st,
                             const void* x_dev, const float* G_dev,
                             float* lfreq_dev, float* lrate_dev, double* totals_dev,
@@ -233,10 +235,10 @@ cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st,
  * same arguments minus the workspace and uses a scratch array compiled into
  * the library instead (4 MiB per GPU, reserved on every GPU that loads the
  * library until the process exits).  It allocates nothing.
- *   Limit: L * 2 * B * H (head slices) <= 512 when dG_dev is given (one 8 KiB
- *   dG partial per slice, d_head = 128, g = 16); larger requests return
- *   CG_ERR_TOO_LARGE before anything is enqueued.  Without dG_dev no scratch is
- *   used and there is no limit.
+ *   Limit: one dG partial of d_head * 16 fp32 per head slice must fit the
+ *   4 MiB array, i.e. L * 2 * B * H <= 512 at d_head = 128 (1024 at 64) when
+ *   dG_dev is given; larger requests return CG_ERR_TOO_LARGE before anything is
+ *   enqueued.  Without dG_dev no scratch is used and there is no limit.
  *   Set-up: the first call on a device looks up the scratch array's device
  *   address (cudaGetSymbolAddress) with that device current; make that first
  *   call before any stream capture.

@@ -58,21 +58,10 @@ cg_status check_range(const cg_kv_desc* kv, const cg_codec_desc* c, int t0, int 
   return CG_OK;
 }
 
-int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
 
 KvGeom geom(const cg_kv_desc* kv) { return KvGeom{kv->layers, kv->batch, kv->heads, kv->tokens, kv->d_head}; }
 
 thread_local cudaError_t t_last_cuda = cudaSuccess;
-
-cg_status from_cuda(cudaError_t e) {
-  if (e == cudaSuccess) return CG_OK;
-  t_last_cuda = e;
-  return CG_ERR_CUDA;
-}
 
 // Device address of the status word on the current device (looked up once
 // per device; a host-side symbol is not a device address).
@@ -91,6 +80,19 @@ unsigned int* status_word() {
 }  // namespace
 
 namespace cg {
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    n = 0;
+  return n > 0 ? n : 148;
+}
+
+cg_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return CG_OK;
+  t_last_cuda = e;
+  return CG_ERR_CUDA;
+}
+
 // Device address of the status word (for entry points defined in other files).
 unsigned int* device_status_word() { return status_word(); }
 
@@ -100,7 +102,6 @@ cg_status validate_stats(const cg_kv_desc* kv, const cg_stats_desc* st) {
   if (s != CG_OK) return s;
   if (!st) return CG_ERR_INVALID;
   if (st->tb != 16) return CG_ERR_UNSUPPORTED;
-  if (kv->d_head != 128 || kv->tokens % 128 != 0) return CG_ERR_UNSUPPORTED;
   if (st->g != 0 && st->g != 16) return CG_ERR_UNSUPPORTED;
   if (!(st->tau > 0.0f)) return CG_ERR_INVALID;
   return CG_OK;

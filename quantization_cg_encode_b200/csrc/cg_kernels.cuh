@@ -38,6 +38,13 @@ cudaError_t launch_fullhead(const CodecArgs& a, bool encode, int num_sms, cudaSt
 uint64_t spectral_workspace_bytes(const KvGeom& k, bool want_grad);
 unsigned int* device_status_word();
 cg_status validate_stats(const cg_kv_desc* kv, const cg_stats_desc* st);
+cudaError_t launch_spectral_generic(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f,
+                                    float lambda_r, float tau, float* lfreq, float* lrate, float* dg_part,
+                                    int num_sms, cudaStream_t st);
+// SM count of the current device, and the C-ABI status of a CUDA error (recorded
+// for cg_last_cuda_error), shared by the entry points.
+int num_sms();
+cg_status from_cuda(cudaError_t e);
 cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f, float lambda_r,
                             float tau, float* lfreq, float* lrate, double* totals, float* dG, void* workspace,
                             unsigned int* status, int num_sms, cudaStream_t st);

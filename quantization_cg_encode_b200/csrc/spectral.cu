@@ -207,6 +207,9 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
     int l, sk, b, h;
     slice_coords(slice, a.k, l, sk, b, h);
     const float* Gp = a.has_g ? a.G + gauge_set(l, sk, h, a.k) * kD * 16 : nullptr;
+    // dG partial of this thread's channel over the slice: each tile's 64 products are
+    // summed afresh and the tile sums added in order, so the rounding grows with
+    // 64 + (tiles per slice) terms rather than with the slice's token count
     float dg[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) dg[j] = 0.0f;
@@ -430,6 +433,9 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
       fence_after();
       {
         const int c = tid & 127, r = c >> 4, th = tid >> 7;  // channel (= TMEM lane), token half
+        float dgt[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) dgt[j] = 0.0f;
         for (int c4 = 2 * th; c4 < 2 * th + 2; ++c4) {
           float v[32];
           ld32(tmem + 128 + 32 * c4 + ((uint32_t)(32 * (warp & 3)) << 16), v);  // dX'^T row c: tokens 32 c4 ..
@@ -455,9 +461,11 @@ __global__ void __launch_bounds__(kSpecThreads, 1) spectral_kernel(SpecArgs a) {
               }
             }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) dg[j] = __fmaf_rn(v[tt], xs[j], dg[j]);
+            for (int j = 0; j < 16; ++j) dgt[j] = __fmaf_rn(v[tt], xs[j], dgt[j]);
           }
         }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) dg[j] = __fadd_rn(dg[j], dgt[j]);
       }
       fence_before();
       named_bar_sync(1, kWorkers);
@@ -518,7 +526,7 @@ __global__ void __launch_bounds__(1024) spectral_totals_kernel(const float* lfre
 
 // dG[l][s][h] = sum over the batch of the per-slice partials, in batch order.
 __global__ void spectral_dg_reduce_kernel(const float* part, float* dG, KvGeom k) {
-  const long long per = (long long)kD * 16;
+  const long long per = (long long)k.d * 16;
   const long long n = (long long)k.L * 2 * k.H * per;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
     const long long set = e / per, off = e % per;
@@ -530,7 +538,7 @@ __global__ void spectral_dg_reduce_kernel(const float* part, float* dG, KvGeom k
 }
 
 uint64_t spectral_workspace_bytes(const KvGeom& k, bool want_grad) {
-  return want_grad ? (uint64_t)k.slices() * kD * 16 * sizeof(float) : 0;
+  return want_grad ? (uint64_t)k.slices() * k.d * 16 * sizeof(float) : 0;
 }
 
 cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f, float lambda_r,
@@ -553,12 +561,18 @@ cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const fl
   a.lrate = lrate;
   a.dg_part = reinterpret_cast<float*>(workspace);
   a.status = status;
-  cudaError_t e = cudaFuncSetAttribute(spectral_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpecSmem);
-  if (e != cudaSuccess) return e;
-  const long long slices = k.slices();
-  const int grid = (int)(slices < num_sms ? slices : num_sms);
-  spectral_kernel<<<grid, kSpecThreads, kSpecSmem, st>>>(a);
-  e = cudaGetLastError();
+  cudaError_t e;
+  if (k.d == kD && k.T % kTile == 0) {
+    e = cudaFuncSetAttribute(spectral_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpecSmem);
+    if (e != cudaSuccess) return e;
+    const long long slices = k.slices();
+    const int grid = (int)(slices < num_sms ? slices : num_sms);
+    spectral_kernel<<<grid, kSpecThreads, kSpecSmem, st>>>(a);
+    e = cudaGetLastError();
+  } else {  // other head widths and token counts: the CUDA-core kernel
+    e = launch_spectral_generic(k, x_fp32, x, G, lambda_f, lambda_r, tau, lfreq, lrate, dG ? a.dg_part : nullptr,
+                                num_sms, st);
+  }
   if (e != cudaSuccess) return e;
   spectral_totals_kernel<<<1, 1024, 0, st>>>(lfreq, lrate, (long long)nblk, lambda_f, lambda_r, totals);
   e = cudaGetLastError();

@@ -7,10 +7,9 @@
 
 namespace {
 
-// One dG partial (d_head x g fp32 = 8 KiB) per head slice.
-constexpr uint64_t kPartialBytes = 128ull * 16ull * sizeof(float);
-constexpr uint64_t kMaxSlices = 512;
-constexpr uint64_t kScratchBytes = kMaxSlices * kPartialBytes;  // 4 MiB
+// One dG partial (d_head x g fp32: 8 KiB at d_head = 128, 4 KiB at 64) per
+// head slice: 512 slices at d_head = 128, 1024 at 64.
+constexpr uint64_t kScratchBytes = 4ull << 20;  // 4 MiB
 
 // Reserved on every device that loads the library, for the life of the process.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -60,10 +59,7 @@ extern "C" cg_status cg_spectral_stats_noalloc(const cg_kv_desc* kv, const cg_st
   }
   unsigned int* status = cg::device_status_word();
   if (!status) return CG_ERR_CUDA;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const cudaError_t e = cg::launch_spectral(k, st->x_is_fp32, x_dev, G_dev, st->lambda_f, st->lambda_r, st->tau,
-                                            lfreq_dev, lrate_dev, totals_dev, dG_dev, scratch, status, sms,
-                                            (cudaStream_t)stream);
-  return e == cudaSuccess ? CG_OK : CG_ERR_CUDA;
+  return cg::from_cuda(cg::launch_spectral(k, st->x_is_fp32, x_dev, G_dev, st->lambda_f, st->lambda_r, st->tau,
+                                           lfreq_dev, lrate_dev, totals_dev, dG_dev, scratch, status, cg::num_sms(),
+                                           (cudaStream_t)stream));
 }
