@@ -308,18 +308,21 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
     const int valid = min(C::TILES, (a.nt - C::UNIT * cur.bq) / 16) - tq * BPW;  // this warp's tiles in range
 
     mbar_wait(&full[s], phase, a.status);
-    // each block's fragments go straight into its MMAs (two terms, two n-halves)
+    // Every block of the stage is computed whether or not its tile lies inside
+    // [t0, t0 + nt) (rows past the range are still inside the stage buffer); only
+    // the stores are predicated.  With no branch per block the compiler can
+    // interleave the eight blocks' dependency chains.
+    // Each block's fragments go straight into its MMAs (two terms, two n-halves).
     float acc[BPW][2][4];
 #pragma unroll
     for (int j = 0; j < BPW; ++j) {
-      if (j < valid) {
-        uint32_t afr[4];
-        ldmatrix_x4(afr, xs_lane + s * C::XBYTES + j * 2048);
+      if (j >= valid) continue;
+      uint32_t afr[4];
+      ldmatrix_x4(afr, xs_lane + s * C::XBYTES + j * 2048);
 #pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-          mma_bf16_16816_z(acc[j][nh], afr, bl[nh][0], bl[nh][1]);
-          mma_bf16_16816(acc[j][nh], afr, bh[nh][0], bh[nh][1]);
-        }
+      for (int nh = 0; nh < 2; ++nh) {
+        mma_bf16_16816_z(acc[j][nh], afr, bl[nh][0], bl[nh][1]);
+        mma_bf16_16816(acc[j][nh], afr, bh[nh][0], bh[nh][1]);
       }
     }
     // the stage is in registers: release it (the last warp refills the slot)
@@ -336,15 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
     float mn = 0.0f, mx = 0.0f;
 #pragma unroll
     for (int j = 0; j < BPW; ++j) {
-      if (j < valid) {
-        const float* v0 = acc[j][0];
-        const float* v1 = acc[j][1];
-        const float bmn = redux_min(min3f(min3f(v0[0], v0[1], v0[2]), min3f(v0[3], v1[0], v1[1]), fminf(v1[2], v1[3])));
-        const float bmx = redux_max(max3f(max3f(v0[0], v0[1], v0[2]), max3f(v0[3], v1[0], v1[1]), fmaxf(v1[2], v1[3])));
-        if (jl == j) {
-          mn = bmn;
-          mx = bmx;
-        }
+      const float* v0 = acc[j][0];
+      const float* v1 = acc[j][1];
+      const float bmn = redux_min(min3f(min3f(v0[0], v0[1], v0[2]), min3f(v0[3], v1[0], v1[1]), fminf(v1[2], v1[3])));
+      const float bmx = redux_max(max3f(max3f(v0[0], v0[1], v0[2]), max3f(v0[3], v1[0], v1[1]), fmaxf(v1[2], v1[3])));
+      if (jl == j) {
+        mn = bmn;
+        mx = bmx;
       }
     }
     mn = __fadd_rn(mn, 0.0f);  // a zero extreme is +0
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
                             : nullptr;
 #pragma unroll
     for (int j = 0; j < BPW; ++j) {
-      if (j >= valid) continue;
+      const bool ok = j < valid;
       const float nz = __shfl_sync(0xffffffffu, nzf, j);
       const float iv = __shfl_sync(0xffffffffu, inv, j);
       const f2_t nz2 = f2_make(nz, nz), iv2 = f2_make(iv, iv), mg2 = f2_make(kMagic, kMagic);
@@ -392,9 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
         rb[2 * k] = __float_as_uint(lo);
         rb[2 * k + 1] = __float_as_uint(hi);
       }
-      store_rows<BITS>(blk0 + j * (C::NG * 32 * BITS), g, c, chunk4<BITS>(rb[0], rb[1], rb[2], rb[3]),
-                       chunk4<BITS>(rb[4], rb[5], rb[6], rb[7]));
-      if (grow0) {
+      const uint32_t v0c = chunk4<BITS>(rb[0], rb[1], rb[2], rb[3]), v1c = chunk4<BITS>(rb[4], rb[5], rb[6], rb[7]);
+      if (ok) store_rows<BITS>(blk0 + j * (C::NG * 32 * BITS), g, c, v0c, v1c);
+      if (grow0 && ok) {
         float* gr = grow0 + j * 16 * D;
         *reinterpret_cast<float4*>(gr) = make_float4(acc[j][0][0], acc[j][0][1], acc[j][1][0], acc[j][1][1]);
         *reinterpret_cast<float4*>(gr + 8 * D) = make_float4(acc[j][0][2], acc[j][0][3], acc[j][1][2], acc[j][1][3]);
