@@ -252,6 +252,17 @@ cg_status cg_spectral_stats_noalloc(const cg_kv_desc* kv, const cg_stats_desc* s
                                     float* lfreq_dev, float* lrate_dev, double* totals_dev,
                                     float* dG_dev, void* stream);
 
+/* Self-test of the failure reporting (no counterpart in the paper: library
+ * diagnostics).  Enqueues one small kernel that waits, with the library's own
+ * bounded mbarrier wait and a limit of limit_ns nanoseconds (1 .. 2e9), on a
+ * barrier that nothing ever completes.  The wait gives up after the limit, the
+ * kernel writes 0 to *result_dev (1 would mean the wait completed) and ends
+ * normally, and the next cg_sync_status() reports CG_ERR_TIMEOUT.  Nothing
+ * faults or hangs; the device stays usable.
+ *   result_dev  device uint32 (output).
+ * Returns CG_ERR_INVALID for a limit out of range or a null pointer. */
+cg_status cg_selftest_wait_timeout(int64_t limit_ns, uint32_t* result_dev, void* stream);
+
 /* Synchronizes `stream`, then reports (and clears) the device status word:
  * CG_ERR_TIMEOUT if a bounded wait ran out since the last check, CG_ERR_CUDA on
  * a pending CUDA error, else CG_OK. */

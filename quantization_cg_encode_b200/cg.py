@@ -20,8 +20,8 @@ ENGINE_AUTO, ENGINE_CUDA_CORES, ENGINE_CHAIN_TENSOR = 0, 1, 2
 
 # Every symbol include/cg.h declares.
 EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
-           "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_sync_status", "cg_last_cuda_error",
-           "cg_status_string", "cg_version")
+           "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_selftest_wait_timeout", "cg_sync_status",
+           "cg_last_cuda_error", "cg_status_string", "cg_version")
 
 
 class KvDesc(ctypes.Structure):
@@ -76,13 +76,15 @@ def lib():
                                         vp, u64, vp]
         L.cg_spectral_stats_noalloc.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(StatsDesc), vp, vp, vp, vp, vp,
                                                 vp, vp]
+        L.cg_selftest_wait_timeout.argtypes = [ctypes.c_int64, vp, vp]
         L.cg_sync_status.argtypes = [vp]
         L.cg_status_string.argtypes = [ctypes.c_int]
         L.cg_status_string.restype = ctypes.c_char_p
         L.cg_version.restype = ctypes.c_int32
         L.cg_last_cuda_error.restype = ctypes.c_char_p
         for name in ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
-                     "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_sync_status"):
+                     "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_selftest_wait_timeout",
+                     "cg_sync_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -206,6 +208,13 @@ def cg_spectral_stats_noalloc(kvd, st, x, G, lfreq, lrate, totals, dG=None, stre
                                            _ptr(G, torch.float32, "G"), _ptr(lfreq, torch.float32, "lfreq"),
                                            _ptr(lrate, torch.float32, "lrate"), _ptr(totals, torch.float64, "totals", 4),
                                            _ptr(dG, torch.float32, "dG"), _stream(stream)), "cg_spectral_stats_noalloc")
+
+
+def cg_selftest_wait_timeout(limit_ns, result, stream=None):
+    """Enqueue the bounded-wait self-test (see include/cg.h); result is a 1-element
+    int32 CUDA tensor that receives 0 when the wait gave up."""
+    _check(lib().cg_selftest_wait_timeout(int(limit_ns), _ptr(result, torch.int32, "result", 1), _stream(stream)),
+           "cg_selftest_wait_timeout")
 
 
 def cg_sync_status(stream=None):

@@ -166,13 +166,15 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t addr, uint32_t parity
   return done;
 }
 // (The first test needs no clock: the common case is a phase already complete.)
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status) {
+// `limit_ns` is the wall-time bound (kWaitNs unless a caller asks for less).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* status,
+                                          unsigned long long limit_ns = kWaitNs) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(addr, parity)) return true;
-    if ((i & 255u) == 0 && global_ns() - t0 > kWaitNs) {
+    if ((i & 255u) == 0 && global_ns() - t0 > limit_ns) {
       atomicOr(status, kStatusTimeout);
       return false;
     }

@@ -99,3 +99,11 @@ def test_decode_and_build_validation_without_gpu():
     assert L.cg_gauge_build(vp(0x1000), vp(0x1000), 4, 16, None) == cg.CG_ERR_INVALID   # aliasing
     assert L.cg_gauge_build(vp(0x1000), vp(0x2000), 4, 200, None) == cg.CG_ERR_INVALID  # g too large
     assert L.cg_gauge_build(vp(0x1000), vp(0x2000), 0, 16, None) == cg.CG_OK            # nothing to do
+
+
+def test_selftest_validation_without_gpu():
+    L = cg.lib()
+    vp = ctypes.c_void_p
+    assert L.cg_selftest_wait_timeout(0, vp(0x1000), None) == cg.CG_ERR_INVALID           # no limit
+    assert L.cg_selftest_wait_timeout(3000000000, vp(0x1000), None) == cg.CG_ERR_INVALID  # above 2 s
+    assert L.cg_selftest_wait_timeout(1000000, vp(0), None) == cg.CG_ERR_INVALID          # null result
