@@ -152,6 +152,50 @@ cg_status cg_sizes_for(const cg_kv_desc* kv, const cg_codec_desc* codec, cg_size
  * One thread block per matrix. */
 cg_status cg_gauge_build(const float* A_dev, float* G_dev, int32_t n_mats, int32_t g, void* stream);
 
+/* AdamW hyperparameters (Loshchilov & Hutter 2019, decoupled weight decay).
+ * The pages name AdamW without its settings; torch's defaults are the reading
+ * taken: lr 1e-3, betas (0.9, 0.999), eps 1e-8, weight decay 0.01. */
+typedef struct {
+  float lr;
+  float beta1;
+  float beta2;
+  float eps;
+  float weight_decay;
+} cg_adamw_desc;
+
+/* dL/dA from dL/dG for G = exp(A - A^T), for n_mats independent g x g matrices
+ * (Codec-Gauge, Method: gauge parameterization and gauge training, where the
+ * objective is optimized through exp).  dS = L_exp(S^T, dG), the adjoint of the
+ * Frechet derivative, is the upper-right g x g block of
+ * exp([[S^T, dG], [0, S^T]]) (Van Loan 1978; Higham 2008, section 10.6), and
+ * dA = dS - dS^T.  One thread block per matrix, fp64 internally.
+ *   A_dev, dG_dev (input), dA_dev (output): fp32 [n_mats][g][g], row-major;
+ *   dA_dev may alias neither input.
+ *   g: 2 .. 32 (CG_ERR_UNSUPPORTED above 32). */
+cg_status cg_gauge_grad(const float* A_dev, const float* dG_dev, float* dA_dev, int32_t n_mats, int32_t g,
+                        void* stream);
+
+/* One AdamW step on n fp32 parameters in place (Codec-Gauge, Method: the gauge
+ * is optimized with AdamW).  With t = step (1-based):
+ *   m = b1 m + (1 - b1) grad,  v = b2 v + (1 - b2) grad^2,
+ *   param -= lr (m / (1 - b1^t) / (sqrt(v / (1 - b2^t)) + eps) + wd param).
+ *   param_dev, m_dev, v_dev: fp32 [n] (updated); grad_dev: fp32 [n] (input).
+ *   m and v start at zero before step 1. */
+cg_status cg_adamw_step(float* param_dev, const float* grad_dev, float* m_dev, float* v_dev, int64_t n,
+                        const cg_adamw_desc* hp, int32_t step, void* stream);
+
+/* Uncentered second-moment (Gram) matrices of every channel group
+ * (Codec-Gauge, Experimental setup: the PCA/KLT control uses the uncentered
+ * second-moment eigenbasis at the layer, K/V, head and group granularity):
+ *   gram[l][s][h][r] = sum over b and t in [t0, t0 + nt) of x x^T, x the g-vector
+ *   of group r of token t.
+ *   kv_dev    bf16 [L][2][B][H][T][d] (input)
+ *   gram_dev  fp64 [L][2][H][d/g][g][g] (output, every entry written)
+ *   g: 8, 16 or 32; any t0 and nt inside [0, T].
+ * Sums run in fp64 in a fixed order (one thread block per gauge set). */
+cg_status cg_group_gram(const cg_kv_desc* kv, int32_t g, const void* kv_dev, int32_t t0, int32_t nt, double* gram_dev,
+                        void* stream);
+
 /* Fused gauge + quantize + pack for tokens [t0, t0 + nt) of every
  * (layer, K/V, batch, head)
  * (Codec-Gauge, Figure 1 / Backend compatibility: the gauge is applied at the

@@ -19,7 +19,8 @@ BLOCK_UNIFORM, KIVI = 0, 1
 ENGINE_AUTO, ENGINE_CUDA_CORES, ENGINE_CHAIN_TENSOR = 0, 1, 2
 
 # Every symbol include/cg.h declares.
-EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
+EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_gauge_grad", "cg_adamw_step", "cg_group_gram", "cg_encode",
+           "cg_decode", "cg_spectral_workspace_size",
            "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_selftest_wait_timeout", "cg_sync_status",
            "cg_last_cuda_error", "cg_status_string", "cg_version")
 
@@ -45,6 +46,15 @@ class StatsDesc(ctypes.Structure):
                 ("lambda_f", ctypes.c_float), ("lambda_r", ctypes.c_float), ("tau", ctypes.c_float)]
 
 
+class AdamwDesc(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float)]
+
+
+def adamw_desc(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01):
+    return AdamwDesc(lr, beta1, beta2, eps, weight_decay)
+
+
 class CgError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -68,6 +78,9 @@ def lib():
         vp, i32, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint64
         L.cg_sizes_for.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), ctypes.POINTER(Sizes)]
         L.cg_gauge_build.argtypes = [vp, vp, i32, i32, vp]
+        L.cg_gauge_grad.argtypes = [vp, vp, vp, i32, i32, vp]
+        L.cg_adamw_step.argtypes = [vp, vp, vp, vp, ctypes.c_int64, ctypes.POINTER(AdamwDesc), i32, vp]
+        L.cg_group_gram.argtypes = [ctypes.POINTER(KvDesc), i32, vp, i32, i32, vp, vp]
         L.cg_encode.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, i32, i32, vp, vp, vp, vp, vp]
         L.cg_decode.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, vp, vp, i32, i32, vp, vp]
         L.cg_spectral_workspace_size.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(StatsDesc), i32,
@@ -82,7 +95,8 @@ def lib():
         L.cg_status_string.restype = ctypes.c_char_p
         L.cg_version.restype = ctypes.c_int32
         L.cg_last_cuda_error.restype = ctypes.c_char_p
-        for name in ("cg_sizes_for", "cg_gauge_build", "cg_encode", "cg_decode", "cg_spectral_workspace_size",
+        for name in ("cg_sizes_for", "cg_gauge_build", "cg_gauge_grad", "cg_adamw_step", "cg_group_gram",
+                     "cg_encode", "cg_decode", "cg_spectral_workspace_size",
                      "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_selftest_wait_timeout",
                      "cg_sync_status"):
             getattr(L, name).restype = ctypes.c_int
@@ -162,6 +176,33 @@ def cg_gauge_build(A, G, stream=None):
     _check(lib().cg_gauge_build(_ptr(A, torch.float32, "A"), _ptr(G, torch.float32, "G", A.numel()), n, g,
                                 _stream(stream)), "cg_gauge_build")
     return G
+
+
+def cg_gauge_grad(A, dG, dA, stream=None):
+    """dL/dA from dL/dG for G = exp(A - A^T); A, dG, dA fp32 of shape [..., g, g]."""
+    g = A.shape[-1]
+    n = A.numel() // (g * g)
+    _check(lib().cg_gauge_grad(_ptr(A, torch.float32, "A"), _ptr(dG, torch.float32, "dG", A.numel()),
+                               _ptr(dA, torch.float32, "dA", A.numel()), n, g, _stream(stream)), "cg_gauge_grad")
+    return dA
+
+
+def cg_adamw_step(param, grad, m, v, hp, step, stream=None):
+    """One AdamW step in place on fp32 CUDA tensors of equal size (step is 1-based)."""
+    n = param.numel()
+    _check(lib().cg_adamw_step(_ptr(param, torch.float32, "param"), _ptr(grad, torch.float32, "grad", n),
+                               _ptr(m, torch.float32, "m", n), _ptr(v, torch.float32, "v", n), n, ctypes.byref(hp),
+                               int(step), _stream(stream)), "cg_adamw_step")
+
+
+def cg_group_gram(kvd, g, kv, gram, t0=0, nt=None, stream=None):
+    """fp64 Gram matrices [L, 2, H, d/g, g, g] of the groups of tokens [t0, t0 + nt)."""
+    nt = kvd.tokens - t0 if nt is None else nt
+    n = kvd.layers * 2 * kvd.batch * kvd.heads * kvd.tokens * kvd.d_head
+    _check(lib().cg_group_gram(ctypes.byref(kvd), int(g), _ptr(kv, torch.bfloat16, "kv", n), int(t0), int(nt),
+                               _ptr(gram, torch.float64, "gram", kvd.layers * 2 * kvd.heads * kvd.d_head * g),
+                               _stream(stream)), "cg_group_gram")
+    return gram
 
 
 def cg_encode(kvd, codec, kv, G, t0, nt, codes, scales, zeros, gauged=None, stream=None):

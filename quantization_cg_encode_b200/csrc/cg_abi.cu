@@ -131,6 +131,40 @@ cg_status cg_gauge_build(const float* A_dev, float* G_dev, int32_t n_mats, int32
   return from_cuda(launch_gauge_build(A_dev, G_dev, n_mats, g, (cudaStream_t)stream));
 }
 
+cg_status cg_gauge_grad(const float* A_dev, const float* dG_dev, float* dA_dev, int32_t n_mats, int32_t g,
+                        void* stream) {
+  if (n_mats < 0 || g < 2 || g > 128) return CG_ERR_INVALID;
+  if (g > 32) return CG_ERR_UNSUPPORTED;
+  if (n_mats == 0) return CG_OK;
+  if (!A_dev || !dG_dev || !dA_dev || !aligned16(A_dev) || !aligned16(dG_dev) || !aligned16(dA_dev)) return CG_ERR_INVALID;
+  if (dA_dev == A_dev || dA_dev == dG_dev) return CG_ERR_INVALID;
+  return from_cuda(launch_gauge_grad(A_dev, dG_dev, dA_dev, n_mats, g, (cudaStream_t)stream));
+}
+
+cg_status cg_adamw_step(float* param_dev, const float* grad_dev, float* m_dev, float* v_dev, int64_t n,
+                        const cg_adamw_desc* hp, int32_t step, void* stream) {
+  if (n < 0 || !hp || step < 1) return CG_ERR_INVALID;
+  if (!(hp->lr >= 0.0f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
+      !(hp->eps > 0.0f) || !(hp->weight_decay >= 0.0f))
+    return CG_ERR_INVALID;
+  if (n == 0) return CG_OK;
+  if (!param_dev || !grad_dev || !m_dev || !v_dev) return CG_ERR_INVALID;
+  if (!aligned16(param_dev) || !aligned16(grad_dev) || !aligned16(m_dev) || !aligned16(v_dev)) return CG_ERR_INVALID;
+  return from_cuda(launch_adamw(param_dev, grad_dev, m_dev, v_dev, n, hp->lr, hp->beta1, hp->beta2, hp->eps,
+                                hp->weight_decay, step, num_sms(), (cudaStream_t)stream));
+}
+
+cg_status cg_group_gram(const cg_kv_desc* kv, int32_t g, const void* kv_dev, int32_t t0, int32_t nt, double* gram_dev,
+                        void* stream) {
+  cg_status st = check_kv(kv);
+  if (st != CG_OK) return st;
+  if (g <= 0 || kv->d_head % g != 0) return CG_ERR_INVALID;
+  if (g != 8 && g != 16 && g != 32) return CG_ERR_UNSUPPORTED;
+  if (t0 < 0 || nt < 0 || (long long)t0 + nt > kv->tokens) return CG_ERR_INVALID;
+  if (!kv_dev || !gram_dev || !aligned16(kv_dev) || !aligned16(gram_dev)) return CG_ERR_INVALID;
+  return from_cuda(launch_gram(geom(kv), g, (const uint16_t*)kv_dev, gram_dev, t0, nt, (cudaStream_t)stream));
+}
+
 cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec, const void* kv_dev, const float* G_dev, int32_t t0,
                     int32_t nt, uint8_t* codes_dev, void* scales_dev, void* zeros_dev, float* gauged_dev, void* stream) {
   cg_status st = check_codec(kv, codec);

@@ -53,5 +53,9 @@ cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const fl
 // box_rows boxes, 128-byte swizzle); `out` points to a CUtensorMap.
 bool make_tmap_2d_bf16(void* out, const void* base, uint64_t rows, uint64_t cols, int box_cols, int box_rows);
 cudaError_t launch_gauge_build(const float* A, float* G, int n_mats, int g, cudaStream_t st);
+cudaError_t launch_gauge_grad(const float* A, const float* dG, float* dA, int n_mats, int g, cudaStream_t st);
+cudaError_t launch_adamw(float* p, const float* grad, float* m, float* v, long long n, float lr, float b1, float b2,
+                         float eps, float wd, int step, int num_sms, cudaStream_t st);
+cudaError_t launch_gram(const KvGeom& k, int g, const uint16_t* kv, double* gram, int t0, int nt, cudaStream_t st);
 
 }  // namespace cg

@@ -27,23 +27,11 @@ __device__ void smem_matmul(const T* A, const T* B, T* C, int n) {
   }
 }
 
+// E = exp(M) for the n x n matrix M in shared memory (M is overwritten by its
+// scaled copy; W is scratch).  Scaling and squaring with the Taylor core.
 template <typename T>
-__global__ void __launch_bounds__(kBuildThreads) gauge_build_kernel(const float* __restrict__ Ain, float* __restrict__ Gout, int n) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  T* M = reinterpret_cast<T*>(smem_raw);  // scaled skew matrix
-  T* E = M + n * n;                        // Horner accumulator / result
-  T* W = E + n * n;                        // product scratch
-  __shared__ T colsum[128];
-  __shared__ int s_shift;
-
-  const long long base = (long long)blockIdx.x * n * n;
-  const float* A = Ain + base;
-  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
-    const int i = e / n, j = e % n;
-    M[e] = (T)A[i * n + j] - (T)A[j * n + i];
-  }
-  __syncthreads();
-  // ||S||_1 = max column sum of |S|
+__device__ void expm_smem(T* M, T* E, T* W, int n, T* colsum, int* s_shift) {
+  // ||M||_1 = max column sum of |M|
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
     T acc = 0;
     for (int i = 0; i < n; ++i) acc += fabs(M[i * n + j]);
@@ -58,10 +46,10 @@ __global__ void __launch_bounds__(kBuildThreads) gauge_build_kernel(const float*
       nrm *= (T)0.5;
       ++s;
     }
-    s_shift = s;
+    *s_shift = s;
   }
   __syncthreads();
-  const int s = s_shift;
+  const int s = *s_shift;
   const T scale = (T)ldexp(1.0, -s);
   for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
     M[e] *= scale;
@@ -82,10 +70,87 @@ __global__ void __launch_bounds__(kBuildThreads) gauge_build_kernel(const float*
     for (int e = threadIdx.x; e < n * n; e += blockDim.x) E[e] = W[e];
     __syncthreads();
   }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kBuildThreads) gauge_build_kernel(const float* __restrict__ Ain, float* __restrict__ Gout, int n) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T* M = reinterpret_cast<T*>(smem_raw);  // scaled skew matrix
+  T* E = M + n * n;                        // Horner accumulator / result
+  T* W = E + n * n;                        // product scratch
+  __shared__ T colsum[128];
+  __shared__ int s_shift;
+
+  const long long base = (long long)blockIdx.x * n * n;
+  const float* A = Ain + base;
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e % n;
+    M[e] = (T)A[i * n + j] - (T)A[j * n + i];
+  }
+  __syncthreads();
+  expm_smem(M, E, W, n, colsum, &s_shift);
   float* G = Gout + base;
   for (int e = threadIdx.x; e < n * n; e += blockDim.x) G[e] = (float)E[e];
 }
+
+// dL/dA for G = exp(S), S = A - A^T, from dL/dG, one matrix per thread block, in
+// fp64.  The adjoint of the Frechet derivative E -> L_exp(S, E) is
+// F -> L_exp(S^T, F) (Higham, Functions of Matrices, 2008, section 10.6), and
+// L_exp(X, F) is the upper-right block of exp([[X, F], [0, X]]) (Van Loan,
+// "Computing integrals involving the matrix exponential", 1978).  So
+// dS = L_exp(S^T, dG) and dA = dS - dS^T.  L_exp is linear in F: dG is scaled
+// to max |dG| = 1 before the exponential and the result scaled back, so the
+// scaling-and-squaring step count depends on S only.
+__global__ void __launch_bounds__(kBuildThreads) gauge_grad_kernel(const float* __restrict__ Ain,
+                                                                   const float* __restrict__ dGin,
+                                                                   float* __restrict__ dAout, int g) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int n = 2 * g;
+  double* M = reinterpret_cast<double*>(smem_raw);
+  double* E = M + n * n;
+  double* W = E + n * n;
+  __shared__ double colsum[64];
+  __shared__ double dgmax[kBuildThreads / 32];
+  __shared__ int s_shift;
+  const long long base = (long long)blockIdx.x * g * g;
+  const float* A = Ain + base;
+  const float* dG = dGin + base;
+  double mloc = 0.0;
+  for (int e = threadIdx.x; e < g * g; e += blockDim.x) mloc = fmax(mloc, fabs((double)dG[e]));
+  for (int o = 16; o >= 1; o >>= 1) mloc = fmax(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+  if ((threadIdx.x & 31) == 0) dgmax[threadIdx.x >> 5] = mloc;
+  __syncthreads();
+  double c = 0.0;
+  for (int w = 0; w < kBuildThreads / 32; ++w) c = fmax(c, dgmax[w]);
+  const double inv_c = c > 0.0 ? 1.0 / c : 0.0;
+  // M = [[S^T, dG / c], [0, S^T]] with S^T[i][j] = A[j][i] - A[i][j]
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e % n;
+    double v = 0.0;
+    if (i < g && j < g) v = (double)A[j * g + i] - (double)A[i * g + j];
+    else if (i >= g && j >= g) v = (double)A[(j - g) * g + (i - g)] - (double)A[(i - g) * g + (j - g)];
+    else if (i < g && j >= g) v = (double)dG[i * g + (j - g)] * inv_c;
+    M[e] = v;
+  }
+  __syncthreads();
+  expm_smem(M, E, W, n, colsum, &s_shift);
+  float* dA = dAout + base;
+  for (int e = threadIdx.x; e < g * g; e += blockDim.x) {
+    const int i = e / g, j = e % g;
+    dA[e] = (float)(c * (E[i * n + g + j] - E[j * n + g + i]));
+  }
+}
 }  // namespace
+
+cudaError_t launch_gauge_grad(const float* A, const float* dG, float* dA, int n_mats, int g, cudaStream_t st) {
+  if (n_mats == 0) return cudaSuccess;
+  if (g > 32) return cudaErrorInvalidValue;
+  const size_t smem = 3 * (size_t)(2 * g) * (2 * g) * sizeof(double);
+  cudaError_t e = cudaFuncSetAttribute(gauge_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gauge_grad_kernel<<<n_mats, kBuildThreads, smem, st>>>(A, dG, dA, g);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_gauge_build(const float* A, float* G, int n_mats, int g, cudaStream_t st) {
   if (n_mats == 0) return cudaSuccess;
