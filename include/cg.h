@@ -239,6 +239,46 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec,
                     const uint8_t* codes_dev, const void* scales_dev, const void* zeros_dev,
                     const float* G_dev, int32_t t0, int32_t nt, void* kv_out_dev, void* stream);
 
+/* Decode-step attention settings.
+ *   q_heads   query heads Hq, a multiple of the cache's KV heads H with
+ *             Hq / H in {1, 2, 4, 8}; query head j uses KV head j / (Hq / H)
+ *             (grouped-query attention).
+ *   n_tokens  attend to cached tokens [0, n_tokens): a multiple of 16 in [16, T].
+ *   layer0, n_layers  the layers [layer0, layer0 + n_layers) of this call.
+ *   scale     score scale, usually 1 / sqrt(d_head). */
+typedef struct {
+  int32_t q_heads;
+  int32_t n_tokens;
+  int32_t layer0;
+  int32_t n_layers;
+  float scale;
+} cg_attn_desc;
+
+/* Workspace bytes cg_decode_attention needs (host only). */
+cg_status cg_decode_attention_workspace_size(const cg_kv_desc* kv, const cg_attn_desc* at, uint64_t* bytes);
+
+/* One decode step of attention read directly from the encoded cache, the
+ * inverse gauge included (Codec-Gauge, Figure 1 / Backend compatibility: keys
+ * and values are restored with G^T before attention).  For every layer l of
+ * the call, batch b and query head j (KV head h = j / (Hq / H)):
+ *   out = sum_t softmax_t(scale q . k_t) v_t,  t in [0, n_tokens),
+ *   k_t = G_K^T (s q_t + z), v_t = G_V^T (s q_t + z) per 16-channel group,
+ * computed as (G_K q) . y_K,t and G_V^T (sum_t p_t y_V,t): the gauge is applied
+ * to the query and the output instead of every cached token (the same result).
+ *   codec       block-uniform, g = 16, 16 x 16 ranges (range_cols = 16), any
+ *               bits; d_head 64 or 128.
+ *   q_dev       bf16 [n_layers][B][Hq][d] (input)
+ *   codes_dev, scales_dev, zeros_dev, G_dev: the whole encoded cache, as
+ *               cg_encode writes it and cg_decode reads it
+ *   out_dev     fp32 [n_layers][B][Hq][d] (output)
+ *   workspace_dev / workspace_bytes: at least
+ *               cg_decode_attention_workspace_size() (per-chunk partials).
+ * Scores and sums are fp32; softmax uses the max-shifted exponential. */
+cg_status cg_decode_attention(const cg_kv_desc* kv, const cg_codec_desc* codec, const cg_attn_desc* at,
+                              const void* q_dev, const uint8_t* codes_dev, const void* scales_dev,
+                              const void* zeros_dev, const float* G_dev, float* out_dev, void* workspace_dev,
+                              uint64_t workspace_bytes, void* stream);
+
 /* Workspace bytes cg_spectral_stats needs for this shape (host only). */
 cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* st,
                                      int32_t want_grad, uint64_t* bytes);

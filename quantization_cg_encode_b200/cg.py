@@ -20,7 +20,7 @@ ENGINE_AUTO, ENGINE_CUDA_CORES, ENGINE_CHAIN_TENSOR = 0, 1, 2
 
 # Every symbol include/cg.h declares.
 EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_gauge_grad", "cg_adamw_step", "cg_group_gram", "cg_encode",
-           "cg_decode", "cg_spectral_workspace_size",
+           "cg_decode", "cg_decode_attention_workspace_size", "cg_decode_attention", "cg_spectral_workspace_size",
            "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_selftest_wait_timeout", "cg_sync_status",
            "cg_last_cuda_error", "cg_status_string", "cg_version")
 
@@ -55,6 +55,11 @@ def adamw_desc(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01):
     return AdamwDesc(lr, beta1, beta2, eps, weight_decay)
 
 
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("q_heads", ctypes.c_int32), ("n_tokens", ctypes.c_int32), ("layer0", ctypes.c_int32),
+                ("n_layers", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
 class CgError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -83,6 +88,10 @@ def lib():
         L.cg_group_gram.argtypes = [ctypes.POINTER(KvDesc), i32, vp, i32, i32, vp, vp]
         L.cg_encode.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, i32, i32, vp, vp, vp, vp, vp]
         L.cg_decode.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, vp, vp, i32, i32, vp, vp]
+        L.cg_decode_attention_workspace_size.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(AttnDesc),
+                                                         ctypes.POINTER(u64)]
+        L.cg_decode_attention.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), ctypes.POINTER(AttnDesc),
+                                          vp, vp, vp, vp, vp, vp, vp, u64, vp]
         L.cg_spectral_workspace_size.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(StatsDesc), i32,
                                                  ctypes.POINTER(u64)]
         L.cg_spectral_stats.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(StatsDesc), vp, vp, vp, vp, vp, vp,
@@ -96,7 +105,8 @@ def lib():
         L.cg_version.restype = ctypes.c_int32
         L.cg_last_cuda_error.restype = ctypes.c_char_p
         for name in ("cg_sizes_for", "cg_gauge_build", "cg_gauge_grad", "cg_adamw_step", "cg_group_gram",
-                     "cg_encode", "cg_decode", "cg_spectral_workspace_size",
+                     "cg_encode", "cg_decode", "cg_decode_attention_workspace_size", "cg_decode_attention",
+                     "cg_spectral_workspace_size",
                      "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_selftest_wait_timeout",
                      "cg_sync_status"):
             getattr(L, name).restype = ctypes.c_int
@@ -222,6 +232,32 @@ def cg_decode(kvd, codec, codes, scales, zeros, G, t0, nt, kv_out, stream=None):
                            _ptr(scales, torch.float16, "scales", sc), _ptr(zeros, torch.float16, "zeros", sc),
                            _ptr(G, torch.float32, "G", gauge_numel(kvd, codec.g)), int(t0), int(nt), _ptr(kv_out, torch.bfloat16, "kv_out", n),
                            _stream(stream)), "cg_decode")
+
+
+def attn_desc(q_heads, n_tokens, layer0=0, n_layers=1, scale=None, d_head=128):
+    return AttnDesc(q_heads, n_tokens, layer0, n_layers, (1.0 / d_head ** 0.5) if scale is None else scale)
+
+
+def cg_decode_attention_workspace_size(kvd, at):
+    out = ctypes.c_uint64()
+    _check(lib().cg_decode_attention_workspace_size(ctypes.byref(kvd), ctypes.byref(at), ctypes.byref(out)),
+           "cg_decode_attention_workspace_size")
+    return int(out.value)
+
+
+def cg_decode_attention(kvd, codec, at, q, codes, scales, zeros, G, out, workspace, stream=None):
+    """Decode-step attention from the encoded cache: q bf16 [n_layers, B, Hq, d] ->
+    out fp32 [n_layers, B, Hq, d]."""
+    cb, sc = cg_sizes_for(kvd, codec)
+    nq = at.n_layers * kvd.batch * at.q_heads * kvd.d_head
+    _check(lib().cg_decode_attention(ctypes.byref(kvd), ctypes.byref(codec), ctypes.byref(at),
+                                     _ptr(q, torch.bfloat16, "q", nq), _ptr(codes, torch.uint8, "codes", cb),
+                                     _ptr(scales, torch.float16, "scales", sc), _ptr(zeros, torch.float16, "zeros", sc),
+                                     _ptr(G, torch.float32, "G", gauge_numel(kvd, codec.g)),
+                                     _ptr(out, torch.float32, "out", nq), ctypes.c_void_p(workspace.data_ptr()),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "cg_decode_attention")
+    return out
 
 
 def cg_spectral_workspace_size(kvd, st, want_grad):

@@ -244,6 +244,62 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec, const uint
 }
 
 
+namespace {
+cg_status check_attn(const cg_kv_desc* kv, const cg_attn_desc* at) {
+  cg_status s = check_kv(kv);
+  if (s != CG_OK) return s;
+  if (!at) return CG_ERR_INVALID;
+  if (at->q_heads <= 0 || at->q_heads % kv->heads != 0) return CG_ERR_INVALID;
+  const int gq = at->q_heads / kv->heads;
+  if (gq != 1 && gq != 2 && gq != 4 && gq != 8) return CG_ERR_UNSUPPORTED;
+  if (at->n_tokens < 16 || at->n_tokens > kv->tokens || at->n_tokens % 16 != 0) return CG_ERR_INVALID;
+  if (at->layer0 < 0 || at->n_layers < 1 || (long long)at->layer0 + at->n_layers > kv->layers) return CG_ERR_INVALID;
+  if (!(at->scale > 0.0f) || !(at->scale < 3.0e38f)) return CG_ERR_INVALID;
+  return CG_OK;
+}
+}  // namespace
+
+cg_status cg_decode_attention_workspace_size(const cg_kv_desc* kv, const cg_attn_desc* at, uint64_t* bytes) {
+  cg_status s = check_attn(kv, at);
+  if (s != CG_OK) return s;
+  if (!bytes) return CG_ERR_INVALID;
+  *bytes = attn_workspace_bytes(geom(kv), at->q_heads, at->n_layers, at->n_tokens);
+  return CG_OK;
+}
+
+cg_status cg_decode_attention(const cg_kv_desc* kv, const cg_codec_desc* codec, const cg_attn_desc* at,
+                              const void* q_dev, const uint8_t* codes_dev, const void* scales_dev,
+                              const void* zeros_dev, const float* G_dev, float* out_dev, void* workspace_dev,
+                              uint64_t workspace_bytes, void* stream) {
+  cg_status s = check_codec(kv, codec);
+  if (s != CG_OK) return s;
+  s = check_attn(kv, at);
+  if (s != CG_OK) return s;
+  if (codec->mode != CG_QUANT_BLOCK_UNIFORM || codec->g != 16 || codec->range_cols != 16) return CG_ERR_UNSUPPORTED;
+  if (!q_dev || !codes_dev || !scales_dev || !zeros_dev || !G_dev || !out_dev || !workspace_dev) return CG_ERR_INVALID;
+  if (!aligned16(q_dev) || !aligned16(codes_dev) || !aligned16(scales_dev) || !aligned16(zeros_dev) ||
+      !aligned16(G_dev) || !aligned16(out_dev) || !aligned16(workspace_dev))
+    return CG_ERR_INVALID;
+  if (workspace_bytes < attn_workspace_bytes(geom(kv), at->q_heads, at->n_layers, at->n_tokens)) return CG_ERR_INVALID;
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.k = geom(kv);
+  a.bits = codec->bits;
+  a.hq = at->q_heads;
+  a.n_tokens = at->n_tokens;
+  a.l0 = at->layer0;
+  a.n_layers = at->n_layers;
+  a.scale = at->scale;
+  a.q = (const uint16_t*)q_dev;
+  a.codes = codes_dev;
+  a.scales = (const uint16_t*)scales_dev;
+  a.zeros = (const uint16_t*)zeros_dev;
+  a.G = G_dev;
+  a.out = out_dev;
+  a.partial = (float*)workspace_dev;
+  return from_cuda(launch_decode_attention(a, (cudaStream_t)stream));
+}
+
 cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* st, int32_t want_grad, uint64_t* bytes) {
   cg_status s = cg::validate_stats(kv, st);
   if (s != CG_OK) return s;

@@ -49,6 +49,26 @@ cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const fl
                             float tau, float* lfreq, float* lrate, double* totals, float* dG, void* workspace,
                             unsigned int* status, int num_sms, cudaStream_t st);
 
+// Arguments of one decode-attention call, after host validation.
+struct AttnArgs {
+  KvGeom k;
+  int bits;
+  int hq;                 // query heads (a multiple of H)
+  int n_tokens;           // attend to tokens [0, n_tokens), a multiple of 16
+  int l0, n_layers;       // layers [l0, l0 + n_layers)
+  int n_chunks;           // set by the launcher
+  float scale;            // score scale (1/sqrt(d) by default)
+  const uint16_t* q;      // bf16 [n_layers][B][hq][d]
+  const uint8_t* codes;   // whole cache, block-uniform 16 x 16 ranges
+  const uint16_t* scales;
+  const uint16_t* zeros;
+  const float* G;         // fp32 [L][2][H][d/16][16][16]
+  float* out;             // fp32 [n_layers][B][hq][d]
+  float* partial;         // workspace
+};
+uint64_t attn_workspace_bytes(const KvGeom& k, int hq, int n_layers, int n_tokens);
+cudaError_t launch_decode_attention(AttnArgs a, cudaStream_t st);
+
 // 2-D TMA tensor map over a row-major bf16 [rows][cols] array (box_cols x
 // box_rows boxes, 128-byte swizzle); `out` points to a CUtensorMap.
 bool make_tmap_2d_bf16(void* out, const void* base, uint64_t rows, uint64_t cols, int box_cols, int box_rows);

@@ -107,3 +107,19 @@ def test_selftest_validation_without_gpu():
     assert L.cg_selftest_wait_timeout(0, vp(0x1000), None) == cg.CG_ERR_INVALID           # no limit
     assert L.cg_selftest_wait_timeout(3000000000, vp(0x1000), None) == cg.CG_ERR_INVALID  # above 2 s
     assert L.cg_selftest_wait_timeout(1000000, vp(0), None) == cg.CG_ERR_INVALID          # null result
+
+
+def test_attention_validation_without_gpu():
+    L = cg.lib()
+    kvd = cg.kv_desc(2, 1, 2, 512, 128)
+    bad = [cg.AttnDesc(5, 512, 0, 1, 0.1),    # Hq not a multiple of H
+           cg.AttnDesc(6 * 2, 512, 0, 1, 0.1),  # group of 6
+           cg.AttnDesc(4, 500, 0, 1, 0.1),    # n not a multiple of 16
+           cg.AttnDesc(4, 528, 0, 1, 0.1),    # n beyond T
+           cg.AttnDesc(4, 512, 1, 2, 0.1),    # layers beyond L
+           cg.AttnDesc(4, 512, 0, 1, 0.0)]    # scale
+    out = ctypes.c_uint64()
+    codes = [cg.CG_ERR_INVALID, cg.CG_ERR_UNSUPPORTED, cg.CG_ERR_INVALID, cg.CG_ERR_INVALID, cg.CG_ERR_INVALID,
+             cg.CG_ERR_INVALID]
+    for at, want in zip(bad, codes):
+        assert L.cg_decode_attention_workspace_size(ctypes.byref(kvd), ctypes.byref(at), ctypes.byref(out)) == want
