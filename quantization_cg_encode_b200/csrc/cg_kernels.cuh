@@ -38,6 +38,10 @@ cudaError_t launch_fullhead(const CodecArgs& a, bool encode, int num_sms, cudaSt
 uint64_t spectral_workspace_bytes(const KvGeom& k, bool want_grad);
 unsigned int* device_status_word();
 cg_status validate_stats(const cg_kv_desc* kv, const cg_stats_desc* st);
+bool spectral_tmem_supported(const KvGeom& k, int x_fp32);
+cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G, float lambda_f, float lambda_r,
+                                 float tau, float* lfreq, float* lrate, float* dg_part, unsigned int* status,
+                                 int num_sms, cudaStream_t st);
 cudaError_t launch_spectral_generic(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f,
                                     float lambda_r, float tau, float* lfreq, float* lrate, float* dg_part,
                                     int num_sms, cudaStream_t st);

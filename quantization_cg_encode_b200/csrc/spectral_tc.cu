@@ -1,0 +1,535 @@
+// Gauge-training statistics with the gauge folded into the channel DCT, on
+// tcgen05 with tensor memory holding one operand of each GEMM (bf16 input,
+// d_head = 128, whole 128-token tiles).
+//
+// Codec-Gauge, Method (frequency-distribution objective): every 16 x 128 block
+// of X' = G X gets U = C_16 X' C_d^T, L_freq = sum r U^2 / sum U^2 and
+// L_rate = mean log(1 + |U| / tau) (assumed form), and the objective's
+// gradient flows back to the group gauges.
+//
+// Restructured so the channel frequency v is the tensor-memory lane:
+//   U1^T = M x^T with M = C_d blockdiag(G)   (one GEMM per 128-token tile: the
+//        gauge is folded into the DCT matrix; x is bf16, exact, streamed by
+//        TMA; M sits in tensor memory as two bf16 terms, M = M_hi + M_lo to
+//        2^-17, as the A operand),
+// so a thread owning lane v holds its channel-frequency row over the tile's
+// tokens and the 16-point token DCT of every block is local to the thread.
+// With the gradient:
+//   dU1^T[v][t] = sum_u C_16[u][t] dU[v][u]   (thread-local again), written
+//        back into tensor memory as two bf16 terms, and
+//   dM += dU1^T x                             (a second GEMM per tile, A from
+//        tensor memory, x from the same shared-memory stage, MN-major),
+//   dG_r[i][j] = sum_v C_d[v][16 r + i] dM[v][16 r + j]   (once per slice).
+//
+// Roles (one CTA per SM, whole head slices per CTA, so each slice's dG partial
+// is a fixed-order sum): warp 0 streams x tiles (two 16 KB boxes, 128-byte
+// swizzle, no multicast) into a 4-stage ring and stages each slice's G; warp 1
+// allocates tensor memory and issues the MMAs; warps 2..9 (channel quarter =
+// warp mod 4, token half = (warp - 2) / 4) build M, run the token DCT, the
+// statistics and the gradient.  Tensor memory: [0,128) U1^T, [128,256) M,
+// [256,384) dU1^T, [384,512) dM.  Every mbarrier wait is bounded in time.
+#include <cuda.h>
+
+#include "cg_kernels.cuh"
+
+namespace cg {
+
+namespace {
+
+constexpr int kD = 128, kTile = 128, kStages = 4;
+constexpr int kXBytes = kTile * kD * 2;
+constexpr int kWorkerWarps = 8;
+constexpr int kThreads = (2 + kWorkerWarps) * 32;
+constexpr uint32_t kColU = 0, kColM = 128, kColDU = 256, kColDM = 384;
+constexpr int kDmPitch = kD + 1;
+// smem: 1024 align + ring + 2 G + dM staging + reductions + barriers
+constexpr int kSmem = 1024 + kStages * kXBytes + 2 * 8192 + kD * kDmPitch * 4 + 2 * 2 * 4 * 12 * 4 + 256;
+
+// Orthonormal DCT-II coefficients C_16[u][t] for t < 8 (the other half follows
+// from C_16[u][15 - t] = (-1)^u C_16[u][t]): 1/4 for u = 0, else
+// sqrt(1/8) cos(pi (2 t + 1) u / 32), folded onto sqrt(1/8) cos(k pi / 32), 0 <= k <= 16.
+constexpr float kCosPi32[17] = {0.3535533845424652f, 0.3518509268760681f, 0.34675997495651245f, 0.3383294939994812f,
+                                0.3266407549381256f, 0.31180626153945923f, 0.29396888613700867f, 0.2733004689216614f,
+                                0.25f, 0.22429189085960388f, 0.19642373919487f, 0.16666391491889954f,
+                                0.13529902696609497f, 0.10263112932443619f, 0.06897484511137009f, 0.034654293209314346f,
+                                0.0f};
+constexpr float c16_value(int u, int t) {
+  int k = ((2 * t + 1) * u) % 64;  // cos(k pi / 32), period 64
+  if (k > 32) k = 64 - k;          // cos(2 pi - a) = cos a
+  float sg = 1.0f;
+  if (k > 16) {                    // cos(pi - a) = -cos a
+    k = 32 - k;
+    sg = -1.0f;
+  }
+  return u == 0 ? 0.25f : sg * kCosPi32[k];
+}
+struct C16Table {
+  float v[16][8];
+};
+constexpr C16Table make_c16() {
+  C16Table c{};
+  for (int u = 0; u < 16; ++u)
+    for (int t = 0; t < 8; ++t) c.v[u][t] = c16_value(u, t);
+  return c;
+}
+__constant__ C16Table c16t = make_c16();
+
+__device__ __forceinline__ uint64_t kdesc(uint32_t addr) {  // K-major, 128-byte swizzle
+  uint64_t d = (uint64_t)((addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+__device__ __forceinline__ uint64_t mndesc(uint32_t addr) {  // MN-major, 128-byte swizzle, 64-element halves 16 KB apart
+  uint64_t d = (uint64_t)((addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(16384 >> 4) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+constexpr uint32_t idesc(bool b_mn) {  // D fp32, A / B bf16, A from tensor memory, M = N = 128
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+}
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t id, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+      "r"(a_tmem), "l"(bdesc), "r"(id), "r"(acc));
+}
+__device__ __forceinline__ void commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// split fp32 pairs into bf16 hi and lo pairs (x = hi + lo to 2^-17)
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(x0, x1);
+  lo = pack_bf16x2(x0 - bf16lo(hi), x1 - bf16hi(hi));
+}
+__device__ __forceinline__ float dct_coef(int k, int n, int N) {
+  const float a = k == 0 ? sqrtf(1.0f / N) : sqrtf(2.0f / N);
+  return a * cospif((2.0f * n + 1.0f) * k / (2.0f * N));
+}
+
+struct TmArgs {
+  KvGeom k;
+  int has_g, want_grad;
+  float lambda_f, lambda_r, tau;
+  double inv_nblk, inv_ncoef;
+  const float* G;
+  float* lfreq;
+  float* lrate;
+  float* dg_part;
+  unsigned int* status;
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid_constant__ CUtensorMap tmap, TmArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* xs = base;                                            // ring of x tiles
+  float* gs = reinterpret_cast<float*>(xs + kStages * kXBytes);        // 2 x [8][16][16] G
+  float* dms = gs + 2 * 2048;                                          // [128][129] dM staging
+  float* red = dms + kD * kDmPitch;                                    // [2 tile parity][2 half][4 quarter][12]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * 2 * 4 * 12);
+  uint64_t* x_full = bars;
+  uint64_t* x_empty = bars + kStages;
+  uint64_t* g_full = bars + 2 * kStages;       // [2]
+  uint64_t* g_empty = g_full + 2;              // [2]
+  uint64_t* m_full = g_empty + 2;
+  uint64_t* m_empty = m_full + 1;
+  uint64_t* u_full = m_empty + 1;
+  uint64_t* u_empty = u_full + 1;
+  uint64_t* du_full = u_empty + 1;
+  uint64_t* du_empty = du_full + 1;
+  uint64_t* dm_full = du_empty + 1;
+  uint64_t* dm_empty = dm_full + 1;
+  uint64_t* mma_done = dm_empty + 1;
+  uint32_t* tmem_base = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile uint32_t* abort_flag = tmem_base + 1;  // set by the first wait that gives up
+  // After one wait has given up, the later ones are skipped, so a broken
+  // pipeline costs one time limit per role, not one per tile.
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    if (*abort_flag) return;
+    if (!mbar_wait(bar, parity, a.status)) *abort_flag = 1u;
+  };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long slices = a.k.slices();
+  const int tiles = a.k.T / kTile;
+  const int n_my = (int)((slices - blockIdx.x + gridDim.x - 1) / gridDim.x);  // slices of this CTA
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&g_full[s], 1);
+      mbar_init(&g_empty[s], kWorkerWarps);
+    }
+    mbar_init(m_full, kWorkerWarps);
+    mbar_init(m_empty, 1);
+    mbar_init(u_full, 1);
+    mbar_init(u_empty, kWorkerWarps);
+    mbar_init(du_full, kWorkerWarps);
+    mbar_init(du_empty, 1);
+    mbar_init(dm_full, 1);
+    mbar_init(dm_empty, kWorkerWarps);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base)), "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_base;
+
+  if (warp == 0) {
+    // ---------------- producer: G of each slice, x tiles ----------------
+    if (lane == 0) {
+      int i = 0;
+      for (int si = 0; si < n_my; ++si) {
+        const long long slice = blockIdx.x + (long long)si * gridDim.x;
+        if (a.has_g) {
+          const int gb = si & 1;
+          wait(&g_empty[gb], ((uint32_t)(si >> 1) & 1u) ^ 1u);
+          int l, sk, b, h;
+          slice_coords(slice, a.k, l, sk, b, h);
+          mbar_arrive_expect_tx(&g_full[gb], 8192);
+          bulk_g2s(gs + gb * 2048, a.G + gauge_set(l, sk, h, a.k) * 2048, 8192, &g_full[gb]);
+        }
+        for (int j = 0; j < tiles; ++j, ++i) {
+          const int s = i % kStages;
+          wait(&x_empty[s], ((uint32_t)(i / kStages) & 1u) ^ 1u);
+          mbar_arrive_expect_tx(&x_full[s], kXBytes);
+          const int row0 = (int)(slice * a.k.T + (long long)j * kTile);
+          tma_load_2d(xs + s * kXBytes, &tmap, 0, row0, &x_full[s]);
+          tma_load_2d(xs + s * kXBytes + 16384, &tmap, 64, row0, &x_full[s]);
+        }
+      }
+      // Drain: the last copy into every stage and G buffer has landed before the
+      // CTA can exit (immediate unless a wait above gave up).
+      for (int s = 0; s < kStages && s < i; ++s) {
+        const int last = ((i - 1 - s) / kStages) * kStages + s;
+        mbar_wait(&x_full[s], (uint32_t)(last / kStages) & 1u, a.status);
+      }
+      if (a.has_g) {
+        for (int si = n_my - 2 < 0 ? 0 : n_my - 2; si < n_my; ++si)
+          mbar_wait(&g_full[si & 1], (uint32_t)(si >> 1) & 1u, a.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issue (one thread) ----------------
+    // Tile f's forward GEMM is issued as soon as its x stage is loaded and the
+    // workers have read tile f-1's U1, i.e. before tile f-1's backward GEMM, except
+    // at the start of a slice with a gauge: its M is built only after the previous
+    // slice's dG, which needs the previous backward first.
+    if (lane == 0) {
+      const int N = n_my * tiles;
+      int f = 0;  // next forward GEMM to issue
+      auto forward = [&](int t) {
+        const int si = t / tiles, j = t % tiles, s = t % kStages;
+        if (j == 0 && (si == 0 || a.has_g)) wait(m_full, (uint32_t)(a.has_g ? si : 0) & 1u);
+        wait(&x_full[s], (uint32_t)(t / kStages) & 1u);
+        wait(u_empty, ((uint32_t)t & 1u) ^ 1u);
+        fence_after();
+        const uint32_t xa = smem_u32(xs + s * kXBytes);
+        // U1^T[v][t] = sum_c M[v][c] x[t][c]: A = M (tensor memory), B = x (K-major)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t bd = kdesc(xa + (k >> 2) * 16384 + (k & 3) * 32);
+          mma_ts(tmem + kColU, tmem + kColM + 8 * k, bd, idesc(false), k > 0);
+          mma_ts(tmem + kColU, tmem + kColM + 64 + 8 * k, bd, idesc(false), 1);
+        }
+        commit(u_full);
+        if (a.has_g && j == tiles - 1) commit(m_empty);  // this slice's M is no longer read
+      };
+      for (int i = 0; i < N; ++i) {
+        if (f == i) forward(f++);
+        if (f < N && (f % tiles != 0 || !a.has_g)) forward(f++);
+        const int si = i / tiles, j = i % tiles, s = i % kStages;
+        if (a.want_grad) {
+          wait(du_full, (uint32_t)i & 1u);
+          if (j == 0 && si > 0) wait(dm_empty, (uint32_t)(si - 1) & 1u);
+          fence_after();
+          const uint32_t xa = smem_u32(xs + s * kXBytes);
+          // dM[v][c] += sum_t dU1^T[v][t] x[t][c]: A = dU1^T (tensor memory), B = x (MN-major)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t bd = mndesc(xa + k * 2048);
+            mma_ts(tmem + kColDM, tmem + kColDU + 8 * k, bd, idesc(true), (j > 0 || k > 0) ? 1u : 0u);
+            mma_ts(tmem + kColDM, tmem + kColDU + 64 + 8 * k, bd, idesc(true), 1);
+          }
+          commit(du_empty);
+          if (j == tiles - 1) commit(dm_full);
+        }
+        commit(&x_empty[s]);  // tile i's stage: both of its GEMMs have been issued before this commit
+      }
+      commit(mma_done);  // every MMA has completed before tensor memory is freed
+      mbar_wait(mma_done, 0u, a.status);
+    }
+  } else {
+    // ---------------- workers: thread = channel frequency v (tensor-memory lane), token half ----------------
+    const int wq = warp & 3, hf = (warp - 2) >> 2, wid = threadIdx.x - 64;  // wid 0..255
+    const int v = 32 * wq + lane;
+    const uint32_t lrow = (uint32_t)(32 * wq) << 16;
+    const float inv_tau = 1.0f / a.tau;
+    float rad[16];
+    {
+      const float rv = (float)v / (kD - 1);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float ru = (float)u / 15.0f;
+        rad[u] = sqrtf(ru * ru + rv * rv) * 0.70710678118654752f;
+      }
+    }
+    int i = 0;
+    for (int si = 0; si < n_my; ++si) {
+      const long long slice = blockIdx.x + (long long)si * gridDim.x;
+      if (si == 0 || a.has_g) {
+        // M[v][c] = sum_i C_d[v][16 r + i] G_r[i][j] for this thread's 64 channels c = 64 hf ..
+        if (a.has_g) wait(&g_full[si & 1], (uint32_t)(si >> 1) & 1u);
+        if (si > 0) wait(m_empty, (uint32_t)(si - 1) & 1u);
+        __syncwarp();
+        fence_after();
+        const float* G = gs + (si & 1) * 2048;
+#pragma unroll 1
+        for (int r4 = 0; r4 < 4; ++r4) {
+          const int r = 4 * hf + r4;
+          float cd[16];
+#pragma unroll
+          for (int ii = 0; ii < 16; ++ii) cd[ii] = dct_coef(v, 16 * r + ii, kD);
+          float m16[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            float acc = 0.0f;
+            if (a.has_g) {
+#pragma unroll
+              for (int ii = 0; ii < 16; ++ii) acc = __fmaf_rn(cd[ii], G[(r * 16 + ii) * 16 + jj], acc);
+            } else {
+              acc = cd[jj];
+            }
+            m16[jj] = acc;
+          }
+          uint32_t h8[8], l8[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) split2(m16[2 * q], m16[2 * q + 1], h8[q], l8[q]);
+          st8(tmem + lrow + kColM + 8 * r, h8);        // channels 16 r .. 16 r + 15: column pairs 8 r ..
+          st8(tmem + lrow + kColM + 64 + 8 * r, l8);
+        }
+        wait_st();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(m_full);
+          if (a.has_g) mbar_arrive(&g_empty[si & 1]);
+        }
+      }
+      for (int j = 0; j < tiles; ++j, ++i) {
+        // U1^T row v, tokens 64 hf .. 64 hf + 63
+        wait(u_full, (uint32_t)i & 1u);
+        __syncwarp();
+        fence_after();
+        float x[64];
+        ld32(tmem + lrow + kColU + 64 * hf, x);
+        ld32(tmem + lrow + kColU + 64 * hf + 32, x + 32);
+        wait_ld();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(u_empty);
+        // token DCT of the four 16-token blocks (even / odd halves), and this v's share of the sums
+        float part[12];  // per block: sum U^2, sum r U^2, sum log2(1 + |U|/tau)
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          float* col = x + 16 * kb;
+          float sm8[8], df8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            sm8[t] = col[t] + col[15 - t];
+            df8[t] = col[t] - col[15 - t];
+          }
+          float e = 0.0f, f = 0.0f, rr = 0.0f;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            float acc = c16t.v[u][0] * ((u & 1) ? df8[0] : sm8[0]);
+#pragma unroll
+            for (int t = 1; t < 8; ++t) acc = __fmaf_rn(c16t.v[u][t], (u & 1) ? df8[t] : sm8[t], acc);
+            col[u] = acc;  // U[u], in place of the block's column (its inputs live in sm8 / df8)
+            const float e2 = acc * acc;
+            e += e2;
+            f = __fmaf_rn(rad[u], e2, f);
+            rr += __log2f(__fmaf_rn(fabsf(acc), inv_tau, 1.0f));
+          }
+          part[3 * kb] = e;
+          part[3 * kb + 1] = f;
+          part[3 * kb + 2] = rr;
+        }
+#pragma unroll
+        for (int q = 0; q < 12; ++q) {
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) part[q] += __shfl_xor_sync(0xffffffffu, part[q], o);
+        }
+        float* rb = red + ((i & 1) * 2 + hf) * 48;  // [quarter][12] of this tile parity and half
+        if (lane == 0) {
+#pragma unroll
+          for (int q = 0; q < 12; ++q) rb[wq * 12 + q] = part[q];
+        }
+        named_bar_sync(2 + hf, 128);
+        float E[4], F[4], R[4], lf[4];
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          E[kb] = (rb[0 * 12 + 3 * kb] + rb[1 * 12 + 3 * kb]) + (rb[2 * 12 + 3 * kb] + rb[3 * 12 + 3 * kb]);
+          F[kb] = (rb[0 * 12 + 3 * kb + 1] + rb[1 * 12 + 3 * kb + 1]) + (rb[2 * 12 + 3 * kb + 1] + rb[3 * 12 + 3 * kb + 1]);
+          R[kb] = (rb[0 * 12 + 3 * kb + 2] + rb[1 * 12 + 3 * kb + 2]) + (rb[2 * 12 + 3 * kb + 2] + rb[3 * 12 + 3 * kb + 2]);
+          lf[kb] = E[kb] > 0.0f ? F[kb] / E[kb] : 0.0f;
+        }
+        if (wq == 0 && lane == 0) {
+          const long long blk0 = slice * (a.k.T / 16) + (long long)j * 8 + 4 * hf;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            a.lfreq[blk0 + kb] = lf[kb];
+            a.lrate[blk0 + kb] = R[kb] * 0.69314718055994531f / (16.0f * kD);
+          }
+        }
+        if (!a.want_grad) continue;
+        // dL/dU, then dU1^T[v][t] = sum_u C_16[u][t] dU[u], into tensor memory as bf16 hi + lo
+        if (i > 0) wait(du_empty, (uint32_t)(i - 1) & 1u);
+        __syncwarp();
+        fence_after();
+        const float cr = (float)(a.lambda_r * a.inv_ncoef);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          const float cf = E[kb] > 0.0f ? (float)(2.0 * a.lambda_f * a.inv_nblk) / E[kb] : 0.0f;
+          float dU[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float U = x[16 * kb + u];
+            const float sg = U > 0.0f ? 1.0f : (U < 0.0f ? -1.0f : 0.0f);
+            dU[u] = __fmaf_rn(cf * U, rad[u] - lf[kb], cr * sg / (a.tau + fabsf(U)));
+          }
+          float d1[16];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            float ev = 0.0f, od = 0.0f;
+#pragma unroll
+            for (int u = 0; u < 16; u += 2) {
+              ev = __fmaf_rn(c16t.v[u][t], dU[u], ev);
+              od = __fmaf_rn(c16t.v[u + 1][t], dU[u + 1], od);
+            }
+            d1[t] = ev + od;
+            d1[15 - t] = ev - od;
+          }
+          uint32_t h8[8], l8[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) split2(d1[2 * q], d1[2 * q + 1], h8[q], l8[q]);
+          st8(tmem + lrow + kColDU + 32 * hf + 8 * kb, h8);
+          st8(tmem + lrow + kColDU + 64 + 32 * hf + 8 * kb, l8);
+        }
+        wait_st();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(du_full);
+        if (j == tiles - 1) {
+          // dG_r[i][j] = sum_v C_d[v][16 r + i] dM[v][16 r + j] for this slice
+          wait(dm_full, (uint32_t)si & 1u);
+          __syncwarp();
+          fence_after();
+          float dm[64];
+          ld32(tmem + lrow + kColDM + 64 * hf, dm);
+          ld32(tmem + lrow + kColDM + 64 * hf + 32, dm + 32);
+          wait_ld();
+          fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dm_empty);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) dms[v * kDmPitch + 64 * hf + c] = dm[c];
+          named_bar_sync(1, kWorkerWarps * 32);
+          {
+            const int ri = wid >> 1, r = ri >> 4, ii = ri & 15, j0 = 8 * (wid & 1);
+            float acc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+#pragma unroll 4
+            for (int vv = 0; vv < kD; ++vv) {
+              const float c = dct_coef(vv, 16 * r + ii, kD);
+              const float* row = dms + vv * kDmPitch + 16 * r + j0;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) acc[q] = __fmaf_rn(c, row[q], acc[q]);
+            }
+            float* dst = a.dg_part + slice * (long long)kD * 16 + (r * 16 + ii) * 16 + j0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = acc[q];
+          }
+          named_bar_sync(1, kWorkerWarps * 32);  // dms is rewritten at the next slice's end
+        }
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+bool spectral_tmem_supported(const KvGeom& k, int x_fp32) { return !x_fp32 && k.d == kD && k.T % kTile == 0; }
+
+cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G, float lambda_f, float lambda_r,
+                                 float tau, float* lfreq, float* lrate, float* dg_part, unsigned int* status,
+                                 int num_sms, cudaStream_t st) {
+  alignas(64) CUtensorMap tmap;
+  if (!make_tmap_2d_bf16(&tmap, x, (uint64_t)k.slices() * k.T, kD, 64, kTile)) return cudaErrorInvalidValue;
+  TmArgs a;
+  a.k = k;
+  a.has_g = G != nullptr;
+  a.want_grad = dg_part != nullptr;
+  a.lambda_f = lambda_f;
+  a.lambda_r = lambda_r;
+  a.tau = tau;
+  const double nblk = (double)k.slices() * (k.T / 16);
+  a.inv_nblk = 1.0 / nblk;
+  a.inv_ncoef = 1.0 / (nblk * 16.0 * kD);
+  a.G = G;
+  a.lfreq = lfreq;
+  a.lrate = lrate;
+  a.dg_part = dg_part;
+  a.status = status;
+  cudaError_t e = cudaFuncSetAttribute(spectral_tmem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
+  const long long slices = k.slices();
+  const int grid = (int)(slices < num_sms ? slices : num_sms);
+  spectral_tmem_kernel<<<grid, kThreads, kSmem, st>>>(tmap, a);
+  return cudaGetLastError();
+}
+
+}  // namespace cg
