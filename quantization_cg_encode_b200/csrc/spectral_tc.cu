@@ -21,8 +21,9 @@
 //        tensor memory, x from the same shared-memory stage, MN-major),
 //   dG_r[i][j] = sum_v C_d[v][16 r + i] dM[v][16 r + j]   (once per slice).
 //
-// Roles (one CTA per SM, whole head slices per CTA, so each slice's dG partial
-// is a fixed-order sum): warp 0 streams x tiles (two 16 KB boxes, 128-byte
+// With dL/dG (the first kernel below; the statistics-only kernel follows it)
+// the roles are (one CTA per SM, whole head slices per CTA, so each slice's dG
+// partial is a fixed-order sum): warp 0 streams x tiles (two 16 KB boxes, 128-byte
 // swizzle, no multicast) into a 4-stage ring and stages each slice's G; warp 1
 // allocates tensor memory and issues the MMAs; warps 2..9 (channel quarter =
 // warp mod 4, token half = (warp - 2) / 4) build M, run the token DCT, the
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
             sm8[t] = col[t] + col[15 - t];
             df8[t] = col[t] - col[15 - t];
           }
-          float e = 0.0f, f = 0.0f, rr = 0.0f;
+          float e = 0.0f, f = 0.0f, rr = 0.0f, pr = 1.0f;
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             float acc = c16t.v[u][0] * ((u & 1) ? df8[0] : sm8[0]);
@@ -387,7 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
             const float e2 = acc * acc;
             e += e2;
             f = __fmaf_rn(rad[u], e2, f);
-            rr += __log2f(__fmaf_rn(fabsf(acc), inv_tau, 1.0f));
+            if (u & 1) rr += __log2f(pr * __fmaf_rn(fabsf(acc), inv_tau, 1.0f));
+            else pr = __fmaf_rn(fabsf(acc), inv_tau, 1.0f);
           }
           part[3 * kb] = e;
           part[3 * kb + 1] = f;
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
           E[kb] = (rb[0 * 12 + 3 * kb] + rb[1 * 12 + 3 * kb]) + (rb[2 * 12 + 3 * kb] + rb[3 * 12 + 3 * kb]);
           F[kb] = (rb[0 * 12 + 3 * kb + 1] + rb[1 * 12 + 3 * kb + 1]) + (rb[2 * 12 + 3 * kb + 1] + rb[3 * 12 + 3 * kb + 1]);
           R[kb] = (rb[0 * 12 + 3 * kb + 2] + rb[1 * 12 + 3 * kb + 2]) + (rb[2 * 12 + 3 * kb + 2] + rb[3 * 12 + 3 * kb + 2]);
-          lf[kb] = E[kb] > 0.0f ? F[kb] / E[kb] : 0.0f;
+          lf[kb] = E[kb] > 0.0f ? __fdividef(F[kb], E[kb]) : 0.0f;
         }
         if (wq == 0 && lane == 0) {
           const long long blk0 = slice * (a.k.T / 16) + (long long)j * 8 + 4 * hf;
@@ -426,15 +428,16 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
         __syncwarp();
         fence_after();
         const float cr = (float)(a.lambda_r * a.inv_ncoef);
+        const float cf0 = (float)(2.0 * a.lambda_f * a.inv_nblk);
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
-          const float cf = E[kb] > 0.0f ? (float)(2.0 * a.lambda_f * a.inv_nblk) / E[kb] : 0.0f;
+          const float cf = E[kb] > 0.0f ? __fdividef(cf0, E[kb]) : 0.0f;
           float dU[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const float U = x[16 * kb + u];
             const float sg = U > 0.0f ? 1.0f : (U < 0.0f ? -1.0f : 0.0f);
-            dU[u] = __fmaf_rn(cf * U, rad[u] - lf[kb], cr * sg / (a.tau + fabsf(U)));
+            dU[u] = __fmaf_rn(cf * U, rad[u] - lf[kb], __fdividef(cr * sg, a.tau + fabsf(U)));
           }
           float d1[16];
 #pragma unroll
@@ -502,6 +505,272 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
   }
 }
 
+// ---------------------------------------------------------------------------
+// Statistics without dL/dG.  The 128-token tiles of all head slices are split
+// into contiguous ranges, one per CTA (a range may start inside a slice and
+// cross into the next ones, each with its own gauge), instead of whole slices,
+// and U1^T is double-buffered in tensor memory so the GEMM of tile i + 1 runs
+// while the workers take tile i's token DCT and statistics.  Tensor memory:
+// [0,128) M (bf16 hi, lo), [128,256) and [256,384) U1^T.
+namespace {
+
+constexpr uint32_t kFColM = 0, kFColU1 = 128;
+constexpr int kFwdSmem = 1024 + kStages * kXBytes + 2 * 8192 + 2 * 2 * 4 * 12 * 4 + 256;
+
+// Sum of 12 per-lane values over a warp: afterwards lane l holds the total of
+// value l >> 1 (l >> 1 < 12).  Each exchange halves the values a lane carries.
+__device__ __forceinline__ float warp_sum12(const float (&p)[12], int lane) {
+  float a8[8], a4[4], a2[2];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const float lo = p[m], hi = m + 8 < 12 ? p[m + 8] : 0.0f;
+    const bool up = lane & 16;
+    a8[m] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, 16);
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const bool up = lane & 8;
+    a4[m] = (up ? a8[m + 4] : a8[m]) + __shfl_xor_sync(0xffffffffu, up ? a8[m] : a8[m + 4], 8);
+  }
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const bool up = lane & 4;
+    a2[m] = (up ? a4[m + 2] : a4[m]) + __shfl_xor_sync(0xffffffffu, up ? a4[m] : a4[m + 2], 4);
+  }
+  const bool up = lane & 2;
+  float r = (up ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, up ? a2[0] : a2[1], 2);
+  return r + __shfl_xor_sync(0xffffffffu, r, 1);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_constant__ CUtensorMap tmap, TmArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* xs = base;                                      // ring of x tiles
+  float* gs = reinterpret_cast<float*>(xs + kStages * kXBytes);  // 2 x [8][16][16] G
+  float* red = reinterpret_cast<float*>(gs + 2 * 2048);          // [2 tile parity][2 half][4 quarter][12]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * 2 * 4 * 12);
+  uint64_t* x_full = bars;
+  uint64_t* x_empty = bars + kStages;
+  uint64_t* g_full = bars + 2 * kStages;  // [2]
+  uint64_t* g_empty = g_full + 2;         // [2]
+  uint64_t* m_full = g_empty + 2;
+  uint64_t* m_empty = m_full + 1;
+  uint64_t* u_full = m_empty + 1;         // [2]
+  uint64_t* u_empty = u_full + 2;         // [2]
+  uint64_t* mma_done = u_empty + 2;
+  uint32_t* tmem_base = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile uint32_t* abort_flag = tmem_base + 1;
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    if (*abort_flag) return;
+    if (!mbar_wait(bar, parity, a.status)) *abort_flag = 1u;
+  };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles = a.k.T / kTile;
+  const long long total = a.k.slices() * tiles;
+  const long long g0 = total * blockIdx.x / gridDim.x;
+  const int n_t = (int)(total * (blockIdx.x + 1) / gridDim.x - g0);  // tiles of this CTA
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&g_full[s], 1);
+      mbar_init(&g_empty[s], kWorkerWarps);
+      mbar_init(&u_full[s], 1);
+      mbar_init(&u_empty[s], kWorkerWarps);
+    }
+    mbar_init(m_full, kWorkerWarps);
+    mbar_init(m_empty, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base)), "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int ls = -1;
+      for (int i = 0; i < n_t; ++i) {
+        const long long gt = g0 + i;
+        const int j = (int)(gt % tiles);
+        if (a.has_g && (i == 0 || j == 0)) {
+          ++ls;
+          const int gb = ls & 1;
+          wait(&g_empty[gb], ((uint32_t)(ls >> 1) & 1u) ^ 1u);
+          int l, sk, b, h;
+          slice_coords(gt / tiles, a.k, l, sk, b, h);
+          mbar_arrive_expect_tx(&g_full[gb], 8192);
+          bulk_g2s(gs + gb * 2048, a.G + gauge_set(l, sk, h, a.k) * 2048, 8192, &g_full[gb]);
+        }
+        const int s = i % kStages;
+        wait(&x_empty[s], ((uint32_t)(i / kStages) & 1u) ^ 1u);
+        mbar_arrive_expect_tx(&x_full[s], kXBytes);
+        const int row0 = (int)(gt * kTile);
+        tma_load_2d(xs + s * kXBytes, &tmap, 0, row0, &x_full[s]);
+        tma_load_2d(xs + s * kXBytes + 16384, &tmap, 64, row0, &x_full[s]);
+      }
+      for (int s = 0; s < kStages && s < n_t; ++s) {
+        const int last = ((n_t - 1 - s) / kStages) * kStages + s;
+        mbar_wait(&x_full[s], (uint32_t)(last / kStages) & 1u, a.status);
+      }
+      for (int q = ls - 1 < 0 ? 0 : ls - 1; q <= ls; ++q) mbar_wait(&g_full[q & 1], (uint32_t)(q >> 1) & 1u, a.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int lsm = -1;
+      for (int i = 0; i < n_t; ++i) {
+        const long long gt = g0 + i;
+        const int j = (int)(gt % tiles), s = i % kStages, ub = i & 1;
+        if (i == 0 || j == 0) {
+          ++lsm;
+          if (a.has_g || i == 0) wait(m_full, (uint32_t)(a.has_g ? lsm : 0) & 1u);
+        }
+        wait(&x_full[s], (uint32_t)(i / kStages) & 1u);
+        wait(&u_empty[ub], ((uint32_t)(i >> 1) & 1u) ^ 1u);
+        fence_after();
+        const uint32_t xa = smem_u32(xs + s * kXBytes);
+        const uint32_t d = tmem + kFColU1 + 128 * ub;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t bd = kdesc(xa + (k >> 2) * 16384 + (k & 3) * 32);
+          mma_ts(d, tmem + kFColM + 8 * k, bd, idesc(false), k > 0);
+          mma_ts(d, tmem + kFColM + 64 + 8 * k, bd, idesc(false), 1);
+        }
+        commit(&u_full[ub]);
+        commit(&x_empty[s]);
+        if (a.has_g && (j == tiles - 1 || i == n_t - 1)) commit(m_empty);
+      }
+      commit(mma_done);
+      mbar_wait(mma_done, 0u, a.status);
+    }
+  } else {
+    const int wq = warp & 3, hf = (warp - 2) >> 2;
+    const int v = 32 * wq + lane;
+    const uint32_t lrow = (uint32_t)(32 * wq) << 16;
+    const float inv_tau = 1.0f / a.tau;
+    float rad[16];
+    {
+      const float rv = (float)v / (kD - 1);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float ru = (float)u / 15.0f;
+        rad[u] = sqrtf(ru * ru + rv * rv) * 0.70710678118654752f;
+      }
+    }
+    int ls = -1;
+    for (int i = 0; i < n_t; ++i) {
+      const long long gt = g0 + i;
+      const int j = (int)(gt % tiles), ub = i & 1;
+      if (i == 0 || j == 0) ++ls;
+      if ((i == 0 || j == 0) && (a.has_g || i == 0)) {
+        if (a.has_g) wait(&g_full[ls & 1], (uint32_t)(ls >> 1) & 1u);
+        if (a.has_g && ls > 0) wait(m_empty, (uint32_t)(ls - 1) & 1u);
+        __syncwarp();
+        fence_after();
+        const float* G = gs + (ls & 1) * 2048;
+#pragma unroll 1
+        for (int r4 = 0; r4 < 4; ++r4) {
+          const int r = 4 * hf + r4;
+          float cd[16];
+#pragma unroll
+          for (int ii = 0; ii < 16; ++ii) cd[ii] = dct_coef(v, 16 * r + ii, kD);
+          float m16[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            float acc = 0.0f;
+            if (a.has_g) {
+#pragma unroll
+              for (int ii = 0; ii < 16; ++ii) acc = __fmaf_rn(cd[ii], G[(r * 16 + ii) * 16 + jj], acc);
+            } else {
+              acc = cd[jj];
+            }
+            m16[jj] = acc;
+          }
+          uint32_t h8[8], l8[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) split2(m16[2 * q], m16[2 * q + 1], h8[q], l8[q]);
+          st8(tmem + lrow + kFColM + 8 * r, h8);
+          st8(tmem + lrow + kFColM + 64 + 8 * r, l8);
+        }
+        wait_st();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(m_full);
+          if (a.has_g) mbar_arrive(&g_empty[ls & 1]);
+        }
+      }
+      wait(&u_full[ub], (uint32_t)(i >> 1) & 1u);
+      __syncwarp();
+      fence_after();
+      float x[64];
+      ld32(tmem + lrow + kFColU1 + 128 * ub + 64 * hf, x);
+      ld32(tmem + lrow + kFColU1 + 128 * ub + 64 * hf + 32, x + 32);
+      wait_ld();
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&u_empty[ub]);
+      float part[12];
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb) {
+        const float* col = x + 16 * kb;
+        float sm8[8], df8[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          sm8[t] = col[t] + col[15 - t];
+          df8[t] = col[t] - col[15 - t];
+        }
+        float e = 0.0f, f = 0.0f, rr = 0.0f, pr = 1.0f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          float U = c16t.v[u][0] * ((u & 1) ? df8[0] : sm8[0]);
+#pragma unroll
+          for (int t = 1; t < 8; ++t) U = __fmaf_rn(c16t.v[u][t], (u & 1) ? df8[t] : sm8[t], U);
+          const float e2 = U * U;
+          e += e2;
+          f = __fmaf_rn(rad[u], e2, f);
+          if (u & 1) rr += __log2f(pr * __fmaf_rn(fabsf(U), inv_tau, 1.0f));
+          else pr = __fmaf_rn(fabsf(U), inv_tau, 1.0f);
+        }
+        part[3 * kb] = e;
+        part[3 * kb + 1] = f;
+        part[3 * kb + 2] = rr;
+      }
+      const float tot = warp_sum12(part, lane);
+      float* rb = red + ((i & 1) * 2 + hf) * 48;
+      if (!(lane & 1) && (lane >> 1) < 12) rb[wq * 12 + (lane >> 1)] = tot;
+      named_bar_sync(2 + hf, 128);
+      if (wq == 0 && lane < 4) {
+        const int kb = lane;
+        const float E = (rb[0 * 12 + 3 * kb] + rb[1 * 12 + 3 * kb]) + (rb[2 * 12 + 3 * kb] + rb[3 * 12 + 3 * kb]);
+        const float F = (rb[0 * 12 + 3 * kb + 1] + rb[1 * 12 + 3 * kb + 1]) + (rb[2 * 12 + 3 * kb + 1] + rb[3 * 12 + 3 * kb + 1]);
+        const float R = (rb[0 * 12 + 3 * kb + 2] + rb[1 * 12 + 3 * kb + 2]) + (rb[2 * 12 + 3 * kb + 2] + rb[3 * 12 + 3 * kb + 2]);
+        const long long blk = gt * 8 + 4 * hf + kb;
+        a.lfreq[blk] = E > 0.0f ? F / E : 0.0f;
+        a.lrate[blk] = R * 0.69314718055994531f / (16.0f * kD);
+      }
+    }
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
 bool spectral_tmem_supported(const KvGeom& k, int x_fp32) { return !x_fp32 && k.d == kD && k.T % kTile == 0; }
 
 cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G, float lambda_f, float lambda_r,
@@ -524,6 +793,14 @@ cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G,
   a.lrate = lrate;
   a.dg_part = dg_part;
   a.status = status;
+  if (dg_part == nullptr) {  // statistics only: tile-balanced ranges
+    cudaError_t e = cudaFuncSetAttribute(spectral_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmem);
+    if (e != cudaSuccess) return e;
+    const long long tiles = k.slices() * (k.T / kTile);
+    const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+    spectral_fwd_kernel<<<grid, kThreads, kFwdSmem, st>>>(tmap, a);
+    return cudaGetLastError();
+  }
   cudaError_t e = cudaFuncSetAttribute(spectral_tmem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   const long long slices = k.slices();

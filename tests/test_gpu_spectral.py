@@ -131,6 +131,7 @@ def test_stats_window_8b_sampled():
     G = oracle_gauge(synth.gauge_params(L, H, 8, 16, sigma=0.1, seed=3))
     lf, lr, tot, dG = run_stats(kv, G, True, False)
     _, _, _, dG_f = run_stats(kv, G, True, False, lambda_r=0.0)
+    lf0, lr0, tot0, _ = run_stats(kv, G, False, False)  # statistics only: the tile-balanced kernel
     # oracle on a few (l, s, h) slices: per-block values, and dG of those gauge sets
     dG = dG.reshape(L, 2, H, 8, 16, 16)
     dG_f = dG_f.reshape(L, 2, H, 8, 16, 16)
@@ -145,6 +146,8 @@ def test_stats_window_8b_sampled():
         rl, rr = ref["lfreq"].reshape(-1), ref["lrate"].reshape(-1)
         assert np.all(np.abs(lf[base:base + nb] - rl) <= 1e-4 * np.maximum(np.abs(rl), 1e-3))
         assert np.all(np.abs(lr[base:base + nb] - rr) <= 1e-4 * np.maximum(np.abs(rr), 1e-3))
+        assert np.all(np.abs(lf0[base:base + nb] - rl) <= 1e-4 * np.maximum(np.abs(rl), 1e-3))
+        assert np.all(np.abs(lr0[base:base + nb] - rr) <= 1e-4 * np.maximum(np.abs(rr), 1e-3))
         # dG of this gauge set is this slice's partial (B = 1).  The oracle's one-slice call
         # normalizes by its own block count; the window's objective by all blocks of the window,
         # and every term of dL/dG carries 1 / n_blocks, so the slice's share is scaled by
@@ -164,6 +167,24 @@ def test_stats_window_8b_sampled():
     lam_r = float(np.float32(0.02))  # lambda_r crosses the C ABI as fp32
     assert abs(tot[3] - (tot[0] / tot[2] + lam_r * tot[1] / tot[2])) <= 1e-12 * abs(tot[3])
     assert np.isfinite(dG).all()
+    assert np.all(np.abs(tot0 - tot) <= 1e-5 * np.abs(tot))
+
+
+@pytest.mark.parametrize("gauged", [True, False])
+def test_stats_forward_tile_ranges(gauged):
+    """Statistics without dL/dG split the 128-token tiles of all head slices into
+    contiguous ranges, one per CTA: 4 x 2 x 1 x 4 slices of 2048 tokens are 512 tiles
+    over at most 148 CTAs, so ranges start inside a slice, cross slice boundaries
+    (each with its own gauge) and wrap the 4-stage ring.  Every block against the
+    oracle, with a g = 16 gauge and without one."""
+    need_gpu()
+    L, B, H, T, d = 4, 1, 4, 2048, 128
+    kv = synth.kv_cache(L, B, H, T, d, seed=8, device="cuda", n_outliers=4)
+    G = oracle_gauge(synth.gauge_params(L, H, 8, 16, sigma=0.1, seed=8)) if gauged else None
+    lf, lr, tot, _ = run_stats(kv, G, False, False)
+    Gn = G.cpu().numpy().astype(np.float64) if gauged else None
+    ref = sp.spectral_stats(bf16_np(kv), Gn)
+    _check(ref, lf, lr, tot)
 
 
 @pytest.mark.parametrize("want_grad", [False, True])
