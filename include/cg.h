@@ -317,10 +317,12 @@ cg_status cg_spectral_stats(const cg_kv_desc* kv, const cg_stats_desc* st,
  * synchronization is not acceptable) cannot create the workspace that
  * cg_spectral_stats needs for its dL/dG partials.  This entry point takes the
  * same arguments minus the workspace and uses a scratch array compiled into
- * the library instead (4 MiB per GPU, reserved on every GPU that loads the
+ * the library instead (8 MiB per GPU, reserved on every GPU that loads the
  * library until the process exits).  It allocates nothing.
- *   Limit: one dG partial of d_head * 16 fp32 per head slice must fit the
- *   4 MiB array, i.e. L * 2 * B * H <= 512 at d_head = 128 (1024 at 64) when
+ *   Limit: the dG partials, d_head * 16 fp32 per work unit (two units per head
+ *   slice at d_head = 128 with T a multiple of 256, one otherwise), must fit
+ *   the 8 MiB array, i.e. L * 2 * B * H <= 512 at d_head = 128 (1024 when T is
+ *   an odd multiple of 128 or not one of 128) and <= 2048 at d_head = 64, when
  *   dG_dev is given; larger requests return CG_ERR_TOO_LARGE before anything is
  *   enqueued.  Without dG_dev no scratch is used and there is no limit.
  *   Set-up: the first call on a device looks up the scratch array's device

@@ -39,6 +39,7 @@ uint64_t spectral_workspace_bytes(const KvGeom& k, bool want_grad);
 unsigned int* device_status_word();
 cg_status validate_stats(const cg_kv_desc* kv, const cg_stats_desc* st);
 bool spectral_tmem_supported(const KvGeom& k, int x_fp32);
+int spectral_tmem_pieces(const KvGeom& k);
 cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G, float lambda_f, float lambda_r,
                                  float tau, float* lfreq, float* lrate, float* dg_part, unsigned int* status,
                                  int num_sms, cudaStream_t st);

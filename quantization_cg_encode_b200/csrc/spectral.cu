@@ -524,21 +524,25 @@ __global__ void __launch_bounds__(1024) spectral_totals_kernel(const float* lfre
   }
 }
 
-// dG[l][s][h] = sum over the batch of the per-slice partials, in batch order.
-__global__ void spectral_dg_reduce_kernel(const float* part, float* dG, KvGeom k) {
+// dG[l][s][h] = sum over the batch, and over the pieces of each head slice, of
+// the per-piece partials, in (batch, piece) order.
+__global__ void spectral_dg_reduce_kernel(const float* part, float* dG, KvGeom k, int pieces) {
   const long long per = (long long)k.d * 16;
   const long long n = (long long)k.L * 2 * k.H * per;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
     const long long set = e / per, off = e % per;
     const long long h = set % k.H, ls = set / k.H;  // ls = l * 2 + s
     float acc = 0.0f;
-    for (int b = 0; b < k.B; ++b) acc += part[((ls * k.B + b) * k.H + h) * per + off];
+    for (int b = 0; b < k.B; ++b)
+      for (int q = 0; q < pieces; ++q) acc += part[(((ls * k.B + b) * k.H + h) * pieces + q) * per + off];
     dG[e] = acc;
   }
 }
 
+// Partials: one per work unit of the kernel that runs (head slices, or their
+// pieces on the tensor-core path); sized for the larger of the two.
 uint64_t spectral_workspace_bytes(const KvGeom& k, bool want_grad) {
-  return want_grad ? (uint64_t)k.slices() * k.d * 16 * sizeof(float) : 0;
+  return want_grad ? (uint64_t)k.slices() * spectral_tmem_pieces(k) * k.d * 16 * sizeof(float) : 0;
 }
 
 cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f, float lambda_r,
@@ -581,7 +585,8 @@ cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const fl
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (dG) {
-    spectral_dg_reduce_kernel<<<num_sms, 256, 0, st>>>(a.dg_part, dG, k);
+    const int pieces = spectral_tmem_supported(k, x_fp32) ? spectral_tmem_pieces(k) : 1;
+    spectral_dg_reduce_kernel<<<num_sms, 256, 0, st>>>(a.dg_part, dG, k, pieces);
     e = cudaGetLastError();
   }
   return e;

@@ -9,7 +9,7 @@ namespace {
 
 // One dG partial (d_head x g fp32: 8 KiB at d_head = 128, 4 KiB at 64) per
 // head slice: 512 slices at d_head = 128, 1024 at 64.
-constexpr uint64_t kScratchBytes = 4ull << 20;  // 4 MiB
+constexpr uint64_t kScratchBytes = 8ull << 20;  // 8 MiB
 
 // Reserved on every device that loads the library, for the life of the process.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];

@@ -22,7 +22,8 @@
 //   dG_r[i][j] = sum_v C_d[v][16 r + i] dM[v][16 r + j]   (once per slice).
 //
 // With dL/dG (the first kernel below; the statistics-only kernel follows it)
-// the roles are (one CTA per SM, whole head slices per CTA, so each slice's dG
+// the roles are (one CTA per SM; the work unit is half a head slice when the
+// slice has an even number of tiles, else the whole slice, and each unit's dG
 // partial is a fixed-order sum): warp 0 streams x tiles (two 16 KB boxes, 128-byte
 // swizzle, no multicast) into a 4-stage ring and stages each slice's G; warp 1
 // allocates tensor memory and issues the MMAs; warps 2..9 (channel quarter =
@@ -44,7 +45,7 @@ constexpr int kThreads = (2 + kWorkerWarps) * 32;
 constexpr uint32_t kColU = 0, kColM = 128, kColDU = 256, kColDM = 384;
 constexpr int kDmPitch = kD + 1;
 // smem: 1024 align + ring + 2 G + dM staging + reductions + barriers
-constexpr int kSmem = 1024 + kStages * kXBytes + 2 * 8192 + kD * kDmPitch * 4 + 2 * 2 * 4 * 12 * 4 + 256;
+constexpr int kSmem = 1024 + kStages * kXBytes + 2 * 8192 + kD * kDmPitch * 4 + 2 * 2 * 4 * 12 * 4 + 132 * 4 + 256;
 
 // Orthonormal DCT-II coefficients C_16[u][t] for t < 8 (the other half follows
 // from C_16[u][15 - t] = (-1)^u C_16[u][t]): 1/4 for u = 0, else
@@ -130,14 +131,52 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
   hi = pack_bf16x2(x0, x1);
   lo = pack_bf16x2(x0 - bf16lo(hi), x1 - bf16hi(hi));
 }
-__device__ __forceinline__ float dct_coef(int k, int n, int N) {
-  const float a = k == 0 ? sqrtf(1.0f / N) : sqrtf(2.0f / N);
-  return a * cospif((2.0f * n + 1.0f) * k / (2.0f * N));
+// Orthonormal DCT-II C_d[v][c] (d = 128) from cosk[k] = cos(k pi / 256), k = 0..128,
+// a table each CTA fills once: the angle (2 c + 1) v pi / 256 is folded onto [0, pi / 2].
+constexpr int kCosTab = 132;  // 129 entries, padded
+__device__ __forceinline__ float cd_tab(const float* cosk, int v, int c) {
+  int k = ((2 * c + 1) * v) & 511;  // period 2 pi = 512 steps
+  if (k > 256) k = 512 - k;         // cos(2 pi - a) = cos a
+  const float cv = k > 128 ? -cosk[256 - k] : cosk[k];  // cos(pi - a) = -cos a
+  return (v == 0 ? 0.08838834764831845f : 0.125f) * cv;  // sqrt(1/128), sqrt(2/128)
+}
+__device__ __forceinline__ void fill_cos_table(float* cosk, int wid) {
+  if (wid <= 128) cosk[wid] = cospif((float)wid / 256.0f);
+}
+// Channels 16 r .. 16 r + 15 of row v of M = C_d blockdiag(G) (C_d alone without a
+// gauge), M[v][16 r + j] = sum_i C_d[v][16 r + i] G_r[i][j], as bf16 hi / lo pairs.
+__device__ __forceinline__ void m_group(const float* cosk, const float* G, bool has_g, int v, int r, uint32_t (&h8)[8],
+                                        uint32_t (&l8)[8]) {
+  float cd[16], m16[16];
+#pragma unroll
+  for (int ii = 0; ii < 16; ++ii) cd[ii] = cd_tab(cosk, v, 16 * r + ii);
+  if (has_g) {
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) m16[jj] = 0.0f;
+#pragma unroll
+    for (int ii = 0; ii < 16; ++ii) {
+      const float4* row = reinterpret_cast<const float4*>(G + (r * 16 + ii) * 16);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 g = row[q];
+        m16[4 * q] = __fmaf_rn(cd[ii], g.x, m16[4 * q]);
+        m16[4 * q + 1] = __fmaf_rn(cd[ii], g.y, m16[4 * q + 1]);
+        m16[4 * q + 2] = __fmaf_rn(cd[ii], g.z, m16[4 * q + 2]);
+        m16[4 * q + 3] = __fmaf_rn(cd[ii], g.w, m16[4 * q + 3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) m16[jj] = cd[jj];
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) split2(m16[2 * q], m16[2 * q + 1], h8[q], l8[q]);
 }
 
 struct TmArgs {
   KvGeom k;
   int has_g, want_grad;
+  int pieces;  // work units per head slice (dL/dG kernel)
   float lambda_f, lambda_r, tau;
   double inv_nblk, inv_ncoef;
   const float* G;
@@ -156,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
   float* gs = reinterpret_cast<float*>(xs + kStages * kXBytes);        // 2 x [8][16][16] G
   float* dms = gs + 2 * 2048;                                          // [128][129] dM staging
   float* red = dms + kD * kDmPitch;                                    // [2 tile parity][2 half][4 quarter][12]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * 2 * 4 * 12);
+  float* cosk = red + 2 * 2 * 4 * 12;                                  // cos(k pi / 256)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cosk + kCosTab);
   uint64_t* x_full = bars;
   uint64_t* x_empty = bars + kStages;
   uint64_t* g_full = bars + 2 * kStages;       // [2]
@@ -180,9 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
   };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long slices = a.k.slices();
-  const int tiles = a.k.T / kTile;
-  const int n_my = (int)((slices - blockIdx.x + gridDim.x - 1) / gridDim.x);  // slices of this CTA
+  // Work unit: a piece of a head slice, tiles / pieces consecutive 128-token tiles
+  // (half a slice when the tile count is even), each with its own dG partial.
+  const long long units = a.k.slices() * a.pieces;
+  const int tiles = a.k.T / kTile / a.pieces;  // tiles per piece
+  const int n_my = (int)((units - blockIdx.x + gridDim.x - 1) / gridDim.x);  // pieces of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -205,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
     *abort_flag = 0u;
     fence_mbar_init();
   }
+  if (warp >= 2) fill_cos_table(cosk, threadIdx.x - 64);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base)), "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -217,9 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
   if (warp == 0) {
     // ---------------- producer: G of each slice, x tiles ----------------
     if (lane == 0) {
-      int i = 0;
-      for (int si = 0; si < n_my; ++si) {
-        const long long slice = blockIdx.x + (long long)si * gridDim.x;
+      int i = 0, g_issued = 0;
+      for (int si = 0; si < n_my && !*abort_flag; ++si) {
+        const long long unit = blockIdx.x + (long long)si * gridDim.x, slice = unit / a.pieces;
+        const int t0 = (int)(unit % a.pieces) * tiles;  // first tile of the piece within its slice
         if (a.has_g) {
           const int gb = si & 1;
           wait(&g_empty[gb], ((uint32_t)(si >> 1) & 1u) ^ 1u);
@@ -227,12 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
           slice_coords(slice, a.k, l, sk, b, h);
           mbar_arrive_expect_tx(&g_full[gb], 8192);
           bulk_g2s(gs + gb * 2048, a.G + gauge_set(l, sk, h, a.k) * 2048, 8192, &g_full[gb]);
+          g_issued = si + 1;
         }
-        for (int j = 0; j < tiles; ++j, ++i) {
+        for (int j = 0; j < tiles && !*abort_flag; ++j, ++i) {
           const int s = i % kStages;
           wait(&x_empty[s], ((uint32_t)(i / kStages) & 1u) ^ 1u);
           mbar_arrive_expect_tx(&x_full[s], kXBytes);
-          const int row0 = (int)(slice * a.k.T + (long long)j * kTile);
+          const int row0 = (int)(slice * a.k.T + (long long)(t0 + j) * kTile);
           tma_load_2d(xs + s * kXBytes, &tmap, 0, row0, &x_full[s]);
           tma_load_2d(xs + s * kXBytes + 16384, &tmap, 64, row0, &x_full[s]);
         }
@@ -243,10 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
         const int last = ((i - 1 - s) / kStages) * kStages + s;
         mbar_wait(&x_full[s], (uint32_t)(last / kStages) & 1u, a.status);
       }
-      if (a.has_g) {
-        for (int si = n_my - 2 < 0 ? 0 : n_my - 2; si < n_my; ++si)
-          mbar_wait(&g_full[si & 1], (uint32_t)(si >> 1) & 1u, a.status);
-      }
+      for (int si = g_issued - 2 < 0 ? 0 : g_issued - 2; si < g_issued; ++si)
+        mbar_wait(&g_full[si & 1], (uint32_t)(si >> 1) & 1u, a.status);
     }
   } else if (warp == 1) {
     // ---------------- MMA issue (one thread) ----------------
@@ -274,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
         commit(u_full);
         if (a.has_g && j == tiles - 1) commit(m_empty);  // this slice's M is no longer read
       };
-      for (int i = 0; i < N; ++i) {
+      for (int i = 0; i < N && !*abort_flag; ++i) {  // after a wait gave up, nothing more is issued
         if (f == i) forward(f++);
         if (f < N && (f % tiles != 0 || !a.has_g)) forward(f++);
         const int si = i / tiles, j = i % tiles, s = i % kStages;
@@ -315,7 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
     }
     int i = 0;
     for (int si = 0; si < n_my; ++si) {
-      const long long slice = blockIdx.x + (long long)si * gridDim.x;
+      const long long unit = blockIdx.x + (long long)si * gridDim.x, slice = unit / a.pieces;
+      const int t0 = (int)(unit % a.pieces) * tiles;
       if (si == 0 || a.has_g) {
         // M[v][c] = sum_i C_d[v][16 r + i] G_r[i][j] for this thread's 64 channels c = 64 hf ..
         if (a.has_g) wait(&g_full[si & 1], (uint32_t)(si >> 1) & 1u);
@@ -326,24 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
 #pragma unroll 1
         for (int r4 = 0; r4 < 4; ++r4) {
           const int r = 4 * hf + r4;
-          float cd[16];
-#pragma unroll
-          for (int ii = 0; ii < 16; ++ii) cd[ii] = dct_coef(v, 16 * r + ii, kD);
-          float m16[16];
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            float acc = 0.0f;
-            if (a.has_g) {
-#pragma unroll
-              for (int ii = 0; ii < 16; ++ii) acc = __fmaf_rn(cd[ii], G[(r * 16 + ii) * 16 + jj], acc);
-            } else {
-              acc = cd[jj];
-            }
-            m16[jj] = acc;
-          }
           uint32_t h8[8], l8[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) split2(m16[2 * q], m16[2 * q + 1], h8[q], l8[q]);
+          m_group(cosk, G, a.has_g, v, r, h8, l8);
           st8(tmem + lrow + kColM + 8 * r, h8);        // channels 16 r .. 16 r + 15: column pairs 8 r ..
           st8(tmem + lrow + kColM + 64 + 8 * r, l8);
         }
@@ -415,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
           lf[kb] = E[kb] > 0.0f ? __fdividef(F[kb], E[kb]) : 0.0f;
         }
         if (wq == 0 && lane == 0) {
-          const long long blk0 = slice * (a.k.T / 16) + (long long)j * 8 + 4 * hf;
+          const long long blk0 = slice * (a.k.T / 16) + (long long)(t0 + j) * 8 + 4 * hf;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             a.lfreq[blk0 + kb] = lf[kb];
@@ -462,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(du_full);
         if (j == tiles - 1) {
-          // dG_r[i][j] = sum_v C_d[v][16 r + i] dM[v][16 r + j] for this slice
+          // dG_r[i][j] = sum_v C_d[v][16 r + i] dM[v][16 r + j] for this piece
           wait(dm_full, (uint32_t)si & 1u);
           __syncwarp();
           fence_after();
@@ -483,16 +511,16 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
             for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
 #pragma unroll 4
             for (int vv = 0; vv < kD; ++vv) {
-              const float c = dct_coef(vv, 16 * r + ii, kD);
+              const float c = cd_tab(cosk, vv, 16 * r + ii);
               const float* row = dms + vv * kDmPitch + 16 * r + j0;
 #pragma unroll
               for (int q = 0; q < 8; ++q) acc[q] = __fmaf_rn(c, row[q], acc[q]);
             }
-            float* dst = a.dg_part + slice * (long long)kD * 16 + (r * 16 + ii) * 16 + j0;
+            float* dst = a.dg_part + unit * (long long)kD * 16 + (r * 16 + ii) * 16 + j0;
 #pragma unroll
             for (int q = 0; q < 8; ++q) dst[q] = acc[q];
           }
-          named_bar_sync(1, kWorkerWarps * 32);  // dms is rewritten at the next slice's end
+          named_bar_sync(1, kWorkerWarps * 32);  // dms is rewritten at the next piece's end
         }
       }
     }
@@ -515,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
 namespace {
 
 constexpr uint32_t kFColM = 0, kFColU1 = 128;
-constexpr int kFwdSmem = 1024 + kStages * kXBytes + 2 * 8192 + 2 * 2 * 4 * 12 * 4 + 256;
+constexpr int kFwdSmem = 1024 + kStages * kXBytes + 2 * 8192 + 2 * 2 * 4 * 12 * 4 + kCosTab * 4 + 256;
 
 // Sum of 12 per-lane values over a warp: afterwards lane l holds the total of
 // value l >> 1 (l >> 1 < 12).  Each exchange halves the values a lane carries.
@@ -550,7 +578,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
   unsigned char* xs = base;                                      // ring of x tiles
   float* gs = reinterpret_cast<float*>(xs + kStages * kXBytes);  // 2 x [8][16][16] G
   float* red = reinterpret_cast<float*>(gs + 2 * 2048);          // [2 tile parity][2 half][4 quarter][12]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * 2 * 4 * 12);
+  float* cosk = red + 2 * 2 * 4 * 12;                            // cos(k pi / 256)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cosk + kCosTab);
   uint64_t* x_full = bars;
   uint64_t* x_empty = bars + kStages;
   uint64_t* g_full = bars + 2 * kStages;  // [2]
@@ -590,6 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
     *abort_flag = 0u;
     fence_mbar_init();
   }
+  if (warp >= 2) fill_cos_table(cosk, threadIdx.x - 64);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base)), "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -601,8 +631,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
 
   if (warp == 0) {
     if (lane == 0) {
-      int ls = -1;
-      for (int i = 0; i < n_t; ++i) {
+      int ls = -1, issued = 0;
+      for (int i = 0; i < n_t && !*abort_flag; ++i) {  // after a wait gave up, nothing more is issued
         const long long gt = g0 + i;
         const int j = (int)(gt % tiles);
         if (a.has_g && (i == 0 || j == 0)) {
@@ -620,9 +650,12 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
         const int row0 = (int)(gt * kTile);
         tma_load_2d(xs + s * kXBytes, &tmap, 0, row0, &x_full[s]);
         tma_load_2d(xs + s * kXBytes + 16384, &tmap, 64, row0, &x_full[s]);
+        issued = i + 1;
       }
-      for (int s = 0; s < kStages && s < n_t; ++s) {
-        const int last = ((n_t - 1 - s) / kStages) * kStages + s;
+      // Drain: the last copy into every stage and G buffer has landed before the
+      // CTA can exit (immediate unless a wait above gave up).
+      for (int s = 0; s < kStages && s < issued; ++s) {
+        const int last = ((issued - 1 - s) / kStages) * kStages + s;
         mbar_wait(&x_full[s], (uint32_t)(last / kStages) & 1u, a.status);
       }
       for (int q = ls - 1 < 0 ? 0 : ls - 1; q <= ls; ++q) mbar_wait(&g_full[q & 1], (uint32_t)(q >> 1) & 1u, a.status);
@@ -630,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
   } else if (warp == 1) {
     if (lane == 0) {
       int lsm = -1;
-      for (int i = 0; i < n_t; ++i) {
+      for (int i = 0; i < n_t && !*abort_flag; ++i) {  // after a wait gave up, nothing more is issued
         const long long gt = g0 + i;
         const int j = (int)(gt % tiles), s = i % kStages, ub = i & 1;
         if (i == 0 || j == 0) {
@@ -683,24 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
 #pragma unroll 1
         for (int r4 = 0; r4 < 4; ++r4) {
           const int r = 4 * hf + r4;
-          float cd[16];
-#pragma unroll
-          for (int ii = 0; ii < 16; ++ii) cd[ii] = dct_coef(v, 16 * r + ii, kD);
-          float m16[16];
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            float acc = 0.0f;
-            if (a.has_g) {
-#pragma unroll
-              for (int ii = 0; ii < 16; ++ii) acc = __fmaf_rn(cd[ii], G[(r * 16 + ii) * 16 + jj], acc);
-            } else {
-              acc = cd[jj];
-            }
-            m16[jj] = acc;
-          }
           uint32_t h8[8], l8[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) split2(m16[2 * q], m16[2 * q + 1], h8[q], l8[q]);
+          m_group(cosk, G, a.has_g, v, r, h8, l8);
           st8(tmem + lrow + kFColM + 8 * r, h8);
           st8(tmem + lrow + kFColM + 64 + 8 * r, l8);
         }
@@ -772,6 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
 }
 
 bool spectral_tmem_supported(const KvGeom& k, int x_fp32) { return !x_fp32 && k.d == kD && k.T % kTile == 0; }
+int spectral_tmem_pieces(const KvGeom& k) { return (k.d == kD && k.T % (2 * kTile) == 0) ? 2 : 1; }
 
 cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G, float lambda_f, float lambda_r,
                                  float tau, float* lfreq, float* lrate, float* dg_part, unsigned int* status,
@@ -801,10 +819,11 @@ cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G,
     spectral_fwd_kernel<<<grid, kThreads, kFwdSmem, st>>>(tmap, a);
     return cudaGetLastError();
   }
+  a.pieces = spectral_tmem_pieces(k);
   cudaError_t e = cudaFuncSetAttribute(spectral_tmem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  const long long slices = k.slices();
-  const int grid = (int)(slices < num_sms ? slices : num_sms);
+  const long long units = k.slices() * a.pieces;
+  const int grid = (int)(units < num_sms ? units : num_sms);
   spectral_tmem_kernel<<<grid, kThreads, kSmem, st>>>(tmap, a);
   return cudaGetLastError();
 }

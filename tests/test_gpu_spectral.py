@@ -79,10 +79,13 @@ def rate_kink_allowance(x, G, n_blocks_total, lambda_r=0.02, tau=0.04, rel_eps=2
     return 3.0 * np.sqrt(tot2.sum(axis=2))                       # [L, 2, H] (summed over the batch)
 
 
-@pytest.mark.parametrize("want_grad", [False, True])
-def test_stats_bf16_cache_with_gauge(want_grad):
+@pytest.mark.parametrize("want_grad,T", [(False, 256), (True, 256), (True, 384)])
+def test_stats_bf16_cache_with_gauge(want_grad, T):
+    """T = 256: two 128-token tiles per head slice, so the dL/dG kernel's work unit
+    is half a slice (two partials per slice); T = 384: an odd tile count, one unit
+    of three tiles per slice."""
     need_gpu()
-    L, B, H, T, d = 2, 2, 2, 256, 128
+    L, B, H, d = 2, 2, 2, 128
     kv = synth.kv_cache(L, B, H, T, d, seed=4, device="cuda")
     G = oracle_gauge(synth.gauge_params(L, H, 8, 16, sigma=0.1, seed=4))
     lf, lr, tot, dG = run_stats(kv, G, want_grad, False)

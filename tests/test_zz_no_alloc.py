@@ -84,8 +84,8 @@ def test_noalloc_forward_only_and_limit():
     cg.cg_sync_status()
     assert _close(lf2, lf) and _close(lr2, lr) and _close(tot2, tot, floor=0.0)
     # a request needing more scratch than is built in is refused before any launch:
-    # 40 x 2 x 1 x 8 = 640 head slices > 512
-    big = cg.kv_desc(40, 1, 8, 128, 128)
+    # 40 x 2 x 1 x 8 = 640 head slices of 256 tokens (two dG partials of 8 KB each) > 8 MiB
+    big = cg.kv_desc(40, 1, 8, 256, 128)
     stg = cg.StatsDesc(16, 16, 0, 1.0, 0.02, 0.04)
     vp = ctypes.c_void_p
     r = cg.lib().cg_spectral_stats_noalloc(ctypes.byref(big), ctypes.byref(stg), vp(0x10000), vp(0x20000),
