@@ -91,6 +91,26 @@ __device__ __forceinline__ uint32_t stage_release(uint32_t* cnt) {
   asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(smem_u32(cnt)) : "memory");
   return old;
 }
+// Wait for a stage; after one wait in the CTA has given up, the others are
+// skipped (one time limit per CTA).  The flag is read only when the stage is
+// not ready at the first test.
+__device__ __forceinline__ void stage_wait(uint64_t* bar, uint32_t phase, volatile uint32_t* abort_v,
+                                           unsigned int* status) {
+  if (mbar_try_wait(smem_u32(bar), phase)) return;
+  if (*abort_v) return;
+  if (!mbar_wait(bar, phase, status)) *abort_v = 1u;
+}
+// Before the CTA exits, the last load issued into every stage has landed
+// (immediate unless a wait gave up and its stage was skipped).
+__device__ __forceinline__ void drain_stages(uint64_t* full, const uint32_t* ctl, int nst, unsigned int* status) {
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  const int n_iss = (int)ctl[1];
+  for (int st = 0; st < nst && st < n_iss; ++st) {
+    const int u = st + nst * ((n_iss - 1 - st) / nst);  // last unit loaded into stage st
+    mbar_wait(&full[st], (uint32_t)(u / nst) & 1u, status);
+  }
+}
 __device__ __forceinline__ float redux_min(float v) {
   float r;
   asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
@@ -237,6 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
   unsigned char* xs = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(xs + NST * C::XBYTES);
   uint32_t* released = reinterpret_cast<uint32_t*>(full + NST);
+  uint32_t* ctl = released + NST;  // [0] abort flag, [1] units issued
+  volatile uint32_t* abort_v = ctl;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -263,6 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
       mbar_init(&full[st], 1);
       released[st] = 0;
     }
+    ctl[0] = 0u;                                   // set by the first wait that gives up
+    ctl[1] = (uint32_t)(n_units < NST ? n_units : NST);  // units whose loads were issued (a prefix)
     fence_mbar_init();
   }
   __syncthreads();
@@ -307,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
     }
     const int valid = min(C::TILES, (a.nt - C::UNIT * cur.bq) / 16) - tq * BPW;  // this warp's tiles in range
 
-    mbar_wait(&full[s], phase, a.status);
+    stage_wait(&full[s], phase, abort_v, a.status);
     // Every block of the stage is computed whether or not its tile lies inside
     // [t0, t0 + nt) (rows past the range are still inside the stage buffer); only
     // the stores are predicated.  With no branch per block the compiler can
@@ -329,7 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
     __syncwarp();
     if (lane == 0 && stage_release(&released[s]) == kWarps - 1) {
       released[s] = 0;
-      if (q + NST < n_units) issue(s, pre);
+      if (q + NST < n_units && !*abort_v) {  // nothing more is loaded after a wait gave up
+        issue(s, pre);
+        ctl[1] = (uint32_t)(q + NST + 1);  // refills run in unit order (ordered by the release atomics)
+      }
     }
     pre.next(bps);
 
@@ -407,6 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_mma16_kernel(const __grid_
       phase ^= 1u;
     }
   }
+  drain_stages(full, ctl, NST, a.status);
 }
 
 namespace {
@@ -439,6 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma16_kernel(CodecArgs a) 
   unsigned char* cs = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
   uint64_t* full = reinterpret_cast<uint64_t*>(cs + NST * C::CSTAGE);
   uint32_t* released = reinterpret_cast<uint32_t*>(full + NST);
+  uint32_t* ctl = released + NST;  // [0] abort flag, [1] units issued
+  volatile uint32_t* abort_v = ctl;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -480,6 +510,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma16_kernel(CodecArgs a) 
       mbar_init(&full[st], 1);
       released[st] = 0;
     }
+    ctl[0] = 0u;                                   // set by the first wait that gives up
+    ctl[1] = (uint32_t)(n_units < NST ? n_units : NST);  // units whose loads were issued (a prefix)
     fence_mbar_init();
   }
   __syncthreads();
@@ -533,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma16_kernel(CodecArgs a) 
     const long long tile0 = slice * T16 + a.t0 / 16 + (long long)C::TILES * cur.bq + tq * BPW;
     const int sz_off = (int)(sz_start(cur) & 15);
 
-    mbar_wait(&full[s], phase, a.status);
+    stage_wait(&full[s], phase, abort_v, a.status);
     const unsigned char* sbase = cs + s * C::CSTAGE;
     const unsigned char* cblk = sbase + (tq * BPW * C::NG + r) * (32 * BITS);
     const __half* szp = reinterpret_cast<const __half*>(sbase + C::CBYTES + C::CSLACK + sz_off) + tq * BPW * C::NG + r;
@@ -565,7 +597,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma16_kernel(CodecArgs a) 
     __syncwarp();
     if (lane == 0 && stage_release(&released[s]) == kWarps - 1) {
       released[s] = 0;
-      if (q + NST < n_units) issue(s, pre);
+      if (q + NST < n_units && !*abort_v) {  // nothing more is loaded after a wait gave up
+        issue(s, pre);
+        ctl[1] = (uint32_t)(q + NST + 1);  // refills run in unit order (ordered by the release atomics)
+      }
     }
     pre.next(sps);
 
@@ -613,6 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma16_kernel(CodecArgs a) 
       phase ^= 1u;
     }
   }
+  drain_stages(full, ctl, NST, a.status);
 }
 
 namespace {
