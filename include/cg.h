@@ -148,8 +148,10 @@ cg_status cg_sizes_for(const cg_kv_desc* kv, const cg_codec_desc* codec, cg_size
  * missing from the page, which names exp(.) and the skew matrix A - A^T).
  *   A_dev, G_dev : fp32 [n_mats][g][g], row-major, may not alias.
  *   g            : 2 .. 128.
- * fp32 scaling and squaring with a Taylor core; G is orthogonal to about 1e-6.
- * One thread block per matrix. */
+ * Scaling and squaring with a degree-14 Taylor core, in fp64 (above g = 64 the
+ * scaled skew matrix is held in fp32), rounded once to fp32: G is within about
+ * 1e-7 of exp(A - A^T) and orthogonal to about 1e-6.  One thread block per
+ * matrix. */
 cg_status cg_gauge_build(const float* A_dev, float* G_dev, int32_t n_mats, int32_t g, void* stream);
 
 /* AdamW hyperparameters (Loshchilov & Hutter 2019, decoupled weight decay).

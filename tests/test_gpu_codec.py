@@ -127,19 +127,22 @@ def test_identity_gauge_is_plain_quantizer_and_degenerate_blocks():
 
 
 def test_gauge_build_group_and_full_head():
-    """cg_gauge_build against the oracle's fp64 exp(A - A^T): fp64 internals for g <= 64
-    (rounded once to fp32), fp32 for g = 128."""
+    """cg_gauge_build against the oracle's fp64 exp(A - A^T), fp64 internals rounded once
+    to fp32 (at g = 128 the scaled skew matrix is held in fp32): max-abs error and
+    orthogonality |G^T G - I| within 1e-5 at every g (1e-6 / 4e-6 for g <= 64), including
+    a g = 128 set whose norm needs several squarings and g = 96 (padded to 128)."""
     need_gpu()
-    for g, sigma, n, tol in [(8, 0.1, 64, 1e-6), (16, 0.1, 512, 1e-6), (32, 0.1, 64, 1e-6), (64, 0.05, 16, 1e-6),
-                             (128, 0.05, 16, 2e-5)]:
+    for g, sigma, n, tol, otol in [(8, 0.1, 64, 1e-6, 4e-6), (16, 0.1, 512, 1e-6, 4e-6), (32, 0.1, 64, 1e-6, 4e-6),
+                                   (64, 0.05, 16, 1e-6, 4e-6), (128, 0.05, 16, 1e-5, 1e-5), (128, 0.5, 4, 1e-5, 1e-5),
+                                   (96, 0.05, 4, 1e-5, 1e-5)]:
         A = torch.randn(n, g, g, generator=torch.Generator().manual_seed(g)) * sigma
         G = torch.empty_like(A).cuda()
         cg.cg_gauge_build(A.cuda(), G)
         Gd = G.cpu().numpy().astype(np.float64)
         Gref = og.gauge_from_A(A.numpy().astype(np.float64))
-        assert np.abs(Gd - Gref).max() < tol, g
+        assert np.abs(Gd - Gref).max() < tol, (g, sigma, np.abs(Gd - Gref).max())
         eye = np.einsum("nji,njk->nik", Gd, Gd)
-        assert np.abs(eye - np.eye(g)).max() < 4 * tol, g
+        assert np.abs(eye - np.eye(g)).max() < otol, (g, sigma, np.abs(eye - np.eye(g)).max())
 
 
 @pytest.mark.slow
