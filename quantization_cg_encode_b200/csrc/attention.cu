@@ -13,11 +13,19 @@
 //
 // Two kernels (flash decoding):
 //   partial: one CTA per (layer, batch, KV head, 256-token chunk) and all query
-//     heads of the GQA group; the chunk's key and value codes, steps and zero
-//     points are staged in shared memory with coalesced 16-byte loads; thread =
-//     token for the scores (q' from shared memory by broadcast), a block
-//     reduction for the chunk's max and exp-sum per head, thread = channel for
-//     the value sums; writes (max, sum, o[d]) per (query head, chunk);
+//     heads of the GQA group.  The chunk's key and value codes, steps and zero
+//     points are staged in shared memory with coalesced 16-byte loads.  Both
+//     contractions run on the warp-level tensor cores (mma.sync m16n8k16,
+//     fp16 operands, fp32 accumulation), one MMA per 16 x 16 range block, with
+//     the codes as exact small integers:
+//       scores  S[t][j] = sum_r s_r (code_r q'_r)[t][j] + z_r sum(q'_r)[j]: A =
+//               the block's key codes, B = q' as fp16 hi + lo terms (scaled per
+//               head by a power of two into fp16's range; about 2^-22 relative),
+//       values  O[c][j] = sum_blocks s (code^T p)[c][j] + z sum_t p[t][j]: A =
+//               the block's value codes transposed, B = the softmax weights as
+//               fp16 hi + lo terms (scaled by 2^12);
+//     the block's step and zero point apply to each MMA result.  Writes (max,
+//     sum, o[d]) per (query head, chunk);
 //   combine: per (layer, batch, query head): merges the chunks' partials with
 //     the usual rescaling, divides by the total, applies G_V^T per group.
 #include "cg_kernels.cuh"
@@ -29,74 +37,55 @@ namespace {
 constexpr int kChunk = 256;  // tokens per CTA
 constexpr int kAttnThreads = 256;
 
-// Code i (0..15) of one 16-code row held in little-endian 32-bit words w.
-template <int BITS>
-__device__ __forceinline__ uint32_t row_code(const uint32_t (&w)[4], int i) {
-  const int bit = i * BITS, wd = bit >> 5, sh = bit & 31;
-  uint32_t v = w[wd] >> sh;
-  if (sh + BITS > 32) v |= w[wd + 1] << (32 - sh);
-  return v & ((1u << BITS) - 1u);
-}
-// The 2*BITS bytes of row `row` of a range block in shared memory.
-template <int BITS>
-__device__ __forceinline__ void load_row(const uint8_t* blk, int row, uint32_t (&w)[4]) {
-  const uint8_t* src = blk + row * 2 * BITS;
-  if constexpr (BITS == 4) {
-    const uint2 v = *reinterpret_cast<const uint2*>(src);
-    w[0] = v.x; w[1] = v.y; w[2] = 0; w[3] = 0;
-  } else if constexpr (BITS == 8) {
-    const uint4 v = *reinterpret_cast<const uint4*>(src);
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-  } else if constexpr (BITS == 2) {
-    w[0] = *reinterpret_cast<const uint32_t*>(src); w[1] = w[2] = w[3] = 0;
-  } else if constexpr (BITS == 3) {  // 6 bytes, 2-byte aligned
-    const uint16_t* h = reinterpret_cast<const uint16_t*>(src);
-    w[0] = h[0] | ((uint32_t)h[1] << 16); w[1] = h[2]; w[2] = w[3] = 0;
-  } else {                            // 6 bits: 12 bytes, 4-byte aligned
-    const uint32_t* u = reinterpret_cast<const uint32_t*>(src);
-    w[0] = u[0]; w[1] = u[1]; w[2] = u[2]; w[3] = 0;
-  }
-}
-// Exact float of a small integer code: the bits 0x4B000000 | c are 2^23 + c.
-__device__ __forceinline__ float code_f(uint32_t c) { return __uint_as_float(0x4B000000u | c) - 8388608.0f; }
-
 }  // namespace
 
 // partial[l][b][hq][chunk] = {m, l, o[D]} in gauge coordinates.
+//
+// MMA columns: for GQ <= 4 one N = 8 tile holds the hi terms of heads 0..3 in
+// columns 0..3 and the lo terms in 4..7 (heads >= GQ are zero); for GQ = 8 a
+// tile of hi terms and a tile of lo terms.  A thread's accumulator columns 2c,
+// 2c+1 are then heads 2c, 2c+1 (hi) or their lo parts, combined by a shuffle.
 template <int D, int BITS, int GQ>
 __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) {
   constexpr int NG = D / 16;
   constexpr int BLK = 32 * BITS;                 // bytes of one 16 x 16 range block
   constexpr int CODE_BYTES = kChunk * D * BITS / 8;
   constexpr int NBLK = kChunk / 16;
+  constexpr int NT = GQ == 8 ? 2 : 1;            // N = 8 tiles per MMA step
+  constexpr float kPScale = 4096.0f;             // p in [0, 1] -> [0, 2^12] for fp16 terms
   extern __shared__ __align__(16) unsigned char smem[];
   uint8_t* kc = smem;                            // key codes of the chunk
-  uint8_t* vc = kc + CODE_BYTES;                 // value codes
-  float* ks = reinterpret_cast<float*>(vc + CODE_BYTES + 16);  // [NBLK][NG] key steps (16 B slack: 2-byte code reads)
+  uint8_t* vc = kc + CODE_BYTES + 16;            // value codes (16 B slack after each)
+  float* ks = reinterpret_cast<float*>(vc + CODE_BYTES + 16);  // [NBLK][NG] key steps
   float* kz = ks + NBLK * NG;
   float* vs = kz + NBLK * NG;
   float* vz = vs + NBLK * NG;
-  float* qp = vz + NBLK * NG;                    // [GQ][D]: q' = G_K q * scale
+  float* qp = vz + NBLK * NG;                    // [GQ][D]: q' = scale * G_K q
   float* qsum = qp + GQ * D;                     // [GQ][NG]: sum of q' over each group
-  float* p = qsum + GQ * NG;                     // [kChunk][GQ]: scores, then exp weights
-  float* red = p + kChunk * GQ;                  // [8 warps][GQ]
+  float* qinv = qsum + GQ * NG;                  // [GQ]: 2^-e_j, the inverse of q''s fp16 scaling
+  float* sc = qinv + 8;                          // [kChunk][GQ]: scores
+  float* psum = sc + kChunk * GQ;                // [NBLK][GQ]: sum of p over each block
+  float* red = psum + NBLK * GQ;                 // [8 warps][GQ]
   float* stat = red + 8 * GQ;                    // [GQ]: chunk max
+  float* po = stat + 8;                          // [2][GQ][D]: value halves (d = 64)
+  uint16_t* pb = reinterpret_cast<uint16_t*>(po + 2 * GQ * D);  // [NCOL][kChunk] fp16 p terms
 
   const int chunk = blockIdx.x;
   const int bh = blockIdx.y;  // b * H + h
   const int lz = blockIdx.z;  // layer index within the call
   const int l = a.l0 + lz;
   const int h = bh % a.k.H, b = bh / a.k.H;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, c = lane & 3;
   const int t0 = chunk * kChunk;
   const int ntok = min(kChunk, a.n_tokens - t0);
-  const int nblk = (ntok + 15) / 16;
+  const int nblk = ntok / 16;  // n_tokens is a multiple of 16
   const long long slice_k = (((long long)l * 2 + 0) * a.k.B + b) * a.k.H + h;
   const long long slice_v = (((long long)l * 2 + 1) * a.k.B + b) * a.k.H + h;
   const long long slice_bytes = (long long)a.k.T * D * BITS / 8;
   const int T16 = a.k.T / 16;
 
-  // stage codes (whole range blocks), steps and zero points
+  // stage codes (whole range blocks), steps and zero points; q' per group
   {
     const uint4* srck = reinterpret_cast<const uint4*>(a.codes + slice_k * slice_bytes + (long long)(t0 / 16) * NG * BLK);
     const uint4* srcv = reinterpret_cast<const uint4*>(a.codes + slice_v * slice_bytes + (long long)(t0 / 16) * NG * BLK);
@@ -112,10 +101,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
       vs[e] = __half2float(__ushort_as_half(a.scales[iv]));
       vz[e] = __half2float(__ushort_as_half(a.zeros[iv]));
     }
-    // q' = scale * G_K q per group, for the GQ query heads of this KV head
     const float* Gk = a.G + gauge_set(l, 0, h, a.k) * NG * 256;
     for (int e = tid; e < GQ * D; e += kAttnThreads) {
-      const int j = e / D, c = e % D, r = c >> 4, i = c & 15;
+      const int j = e / D, cc = e % D, r = cc >> 4, i = cc & 15;
       const uint16_t* qrow = a.q + (((long long)lz * a.k.B + b) * a.hq + h * GQ + j) * D + 16 * r;
       const float* gi = Gk + (r * 16 + i) * 16;
       float acc = 0.0f;
@@ -132,129 +120,253 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
     for (int i = 0; i < 16; ++i) s += q[i];
     qsum[e] = s;
   }
-  __syncthreads();
-
-  // scores, thread = token: sum over groups of s (q' . code) + z sum(q')
-  float sc[GQ];
-  const int t = tid;
-  const bool live = t < ntok;
-  {
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) sc[j] = -INFINITY;
-    if (live) {
-#pragma unroll
-      for (int j = 0; j < GQ; ++j) sc[j] = 0.0f;
-      const int kb = t >> 4, row = t & 15;
-#pragma unroll 1
-      for (int r = 0; r < NG; ++r) {
-        uint32_t w[4];
-        load_row<BITS>(kc + (kb * NG + r) * BLK, row, w);
-        float acc[GQ];
-#pragma unroll
-        for (int j = 0; j < GQ; ++j) acc[j] = 0.0f;
-#pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-          float cf[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) cf[e] = code_f(row_code<BITS>(w, 4 * i4 + e));
-#pragma unroll
-          for (int j = 0; j < GQ; ++j) {
-            const float4 q4 = *reinterpret_cast<const float4*>(qp + j * D + 16 * r + 4 * i4);  // broadcast
-            acc[j] = __fmaf_rn(q4.x, cf[0], acc[j]);
-            acc[j] = __fmaf_rn(q4.y, cf[1], acc[j]);
-            acc[j] = __fmaf_rn(q4.z, cf[2], acc[j]);
-            acc[j] = __fmaf_rn(q4.w, cf[3], acc[j]);
-          }
-        }
-        const float s = ks[kb * NG + r], z = kz[kb * NG + r];
-#pragma unroll
-        for (int j = 0; j < GQ; ++j) sc[j] += __fmaf_rn(s, acc[j], z * qsum[j * NG + r]);
-      }
-    }
-  }
-  // chunk max and exp weights per query head
-  const int warp = tid >> 5, lane = tid & 31;
-#pragma unroll
-  for (int j = 0; j < GQ; ++j) {
-    float m = sc[j];
+  if (warp < GQ) {  // fp16 scaling of head j: max |q'| * 2^e_j in [2^14, 2^15)
+    float m = 0.0f;
+    for (int i = lane; i < D; i += 32) m = fmaxf(m, fabsf(qp[warp * D + i]));
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) red[warp * GQ + j] = m;
-  }
-  __syncthreads();
-  if (tid < GQ) {
-    float m = red[tid];
-    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w * GQ + tid]);
-    stat[tid] = m;
-  }
-  __syncthreads();
-  float ls[GQ];
-#pragma unroll
-  for (int j = 0; j < GQ; ++j) {
-    const float pj = live ? __expf(sc[j] - stat[j]) : 0.0f;
-    p[t * GQ + j] = pj;
-    ls[j] = pj;
-  }
-  __syncthreads();  // red is reused below, p is read by every thread
-#pragma unroll
-  for (int j = 0; j < GQ; ++j) {
-    float s = ls[j];
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) red[warp * GQ + j] = s;
+    int ex = 0;
+    if (m > 0.0f) frexpf(m, &ex);
+    if (lane == 0) qinv[warp] = m > 0.0f ? ldexpf(1.0f, ex - 15) : 1.0f;
   }
   __syncthreads();
 
-  // value sums in gauge coordinates, thread = channel (threads D .. 2D-1 take the
-  // second half of the tokens; their sums are added in a fixed order)
-  float* out = a.partial + ((((long long)lz * a.k.B + b) * a.hq + h * GQ) * a.n_chunks + chunk) * (D + 2);
-  const long long head_stride = (long long)a.n_chunks * (D + 2);
-  constexpr int HALVES = kAttnThreads / D;  // 2 (d = 128) or 4 (d = 64)
-  const int c = tid % D, part = tid / D, r = c >> 4, i = c & 15;
-  float o[GQ];
+  // ---- scores on the tensor cores: warp w takes blocks w and w + 8 ----
+  {
+    // B fragments: column n = g of tile tt holds q'' = q' 2^e of (term, head);
+    // k slots 2c, 2c+1 / 2c+8, 2c+9 are channels 4c, 4c+1 / 4c+2, 4c+3 of the group
+    uint32_t bq[NG][NT][2];
 #pragma unroll
-  for (int j = 0; j < GQ; ++j) o[j] = 0.0f;
-  const int per = (nblk + HALVES - 1) / HALVES;
-  for (int kb = part * per; kb < min(nblk, part * per + per); ++kb) {
-    const uint8_t* blk = vc + (kb * NG + r) * BLK;
-    const float s = vs[kb * NG + r], z = vz[kb * NG + r];
-    float acc[GQ], psum[GQ];
+    for (int tt = 0; tt < NT; ++tt) {
+      const int j = NT == 2 ? g : (g & 3), lo = NT == 2 ? tt : (g >> 2);
+      const bool on = j < GQ;
+      const float sj = on ? 1.0f / qinv[j] : 0.0f;
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) acc[j] = psum[j] = 0.0f;
-#pragma unroll 4
-    for (int row = 0; row < 16; ++row) {
-      const int bit = (row * 16 + i) * BITS;
-      const uint32_t wv = (uint32_t)blk[bit >> 3] | ((uint32_t)blk[(bit >> 3) + 1] << 8);
-      const float cf = code_f((wv >> (bit & 7)) & ((1u << BITS) - 1u));
-      const float* pr = p + (kb * 16 + row) * GQ;  // broadcast
+      for (int r = 0; r < NG; ++r) {
+        float4 q4 = on ? *reinterpret_cast<const float4*>(qp + j * D + 16 * r + 4 * c) : make_float4(0, 0, 0, 0);
+        const float v[4] = {q4.x * sj, q4.y * sj, q4.z * sj, q4.w * sj};
+        __half hv[4];
 #pragma unroll
-      for (int j = 0; j < GQ; ++j) {
-        acc[j] = __fmaf_rn(pr[j], cf, acc[j]);
-        psum[j] += pr[j];
+        for (int e = 0; e < 4; ++e) {
+          const __half hi = __float2half_rn(v[e]);
+          hv[e] = lo ? __float2half_rn(v[e] - __half2float(hi)) : hi;
+        }
+        bq[r][tt][0] = (uint32_t)__half_as_ushort(hv[0]) | ((uint32_t)__half_as_ushort(hv[1]) << 16);
+        bq[r][tt][1] = (uint32_t)__half_as_ushort(hv[2]) | ((uint32_t)__half_as_ushort(hv[3]) << 16);
       }
     }
+    const int bit_g = (16 * g + 4 * c) * BITS, bit_g8 = (16 * (g + 8) + 4 * c) * BITS;
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) o[j] += __fmaf_rn(s, acc[j], z * psum[j]);
-  }
-  // combine the token parts in order through shared memory (p is no longer needed)
-  __syncthreads();
-  float* po = p;  // [HALVES][GQ][D]
+    for (int bi = 0; bi < 2; ++bi) {
+      const int kb = warp + 8 * bi;
+      if (kb >= nblk) continue;  // warp-uniform
+      float acc[NT][4];
 #pragma unroll
-  for (int j = 0; j < GQ; ++j) po[(part * GQ + j) * D + c] = o[j];
-  __syncthreads();
-  if (part == 0) {
+      for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-      float v = po[j * D + c];
-      for (int q2 = 1; q2 < HALVES; ++q2) v += po[(q2 * GQ + j) * D + c];
-      out[j * head_stride + 2 + c] = v;
+        for (int e = 0; e < 4; ++e) acc[tt][e] = 0.0f;
+#pragma unroll
+      for (int r = 0; r < NG; ++r) {
+        const uint8_t* blk = kc + (kb * NG + r) * BLK;
+        uint32_t cv[2];  // rows g, g+8: codes 4c .. 4c+3 (4 BITS bits, low aligned)
+        if constexpr (BITS == 4) {
+          cv[0] = *reinterpret_cast<const uint16_t*>(blk + (bit_g >> 3));
+          cv[1] = *reinterpret_cast<const uint16_t*>(blk + (bit_g8 >> 3));
+        } else if constexpr (BITS == 8) {
+          cv[0] = *reinterpret_cast<const uint32_t*>(blk + (bit_g >> 3));
+          cv[1] = *reinterpret_cast<const uint32_t*>(blk + (bit_g8 >> 3));
+        } else if constexpr (BITS == 2) {
+          cv[0] = blk[bit_g >> 3];
+          cv[1] = blk[bit_g8 >> 3];
+        } else {
+          const uint32_t* w0 = reinterpret_cast<const uint32_t*>(blk) + (bit_g >> 5);
+          const uint32_t* w1 = reinterpret_cast<const uint32_t*>(blk) + (bit_g8 >> 5);
+          cv[0] = __funnelshift_r(w0[0], w0[1], bit_g & 31);
+          cv[1] = __funnelshift_r(w1[0], w1[1], bit_g8 & 31);
+        }
+        uint32_t afr[4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          constexpr uint32_t M = (1u << BITS) - 1u;
+          const uint32_t v = cv[hh];
+          afr[hh] = f16_sub1024(0x64006400u | (v & M) | (((v >> BITS) & M) << 16));
+          afr[2 + hh] = f16_sub1024(0x64006400u | ((v >> (2 * BITS)) & M) | (((v >> (3 * BITS)) & M) << 16));
+        }
+        const float sk = ks[kb * NG + r];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) {
+          float d[4];
+          mma_f16_16816_z(d, afr, bq[r][tt][0], bq[r][tt][1]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[tt][e] = __fmaf_rn(sk, d[e], acc[tt][e]);
+        }
+      }
+      // hi + lo terms; then columns 2c, 2c+1 are heads 2c, 2c+1 (threads c < 2 for GQ <= 4)
+      float sv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if constexpr (NT == 2) {
+          sv[e] = acc[0][e] + acc[1][e];
+        } else {
+          sv[e] = acc[0][e] + __shfl_xor_sync(0xffffffffu, acc[0][e], 2);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 2 * c + (e & 1), t = kb * 16 + g + 8 * (e >> 1);
+        if ((NT == 2 || c < 2) && j < GQ) {
+          float zt = 0.0f;
+#pragma unroll
+          for (int r = 0; r < NG; ++r) zt = __fmaf_rn(kz[kb * NG + r], qsum[j * NG + r], zt);
+          sc[t * GQ + j] = __fmaf_rn(sv[e], qinv[j], zt);
+        }
+      }
     }
   }
-  if (tid < GQ) {
-    float s = 0.0f;
-    for (int w = 0; w < 8; ++w) s += red[w * GQ + tid];
-    out[tid * head_stride + 0] = stat[tid];
-    out[tid * head_stride + 1] = s;
+  __syncthreads();
+
+  // ---- softmax over the chunk, thread = token ----
+  {
+    const int t = tid;
+    const bool live = t < ntok;
+    float sj[GQ];
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+      sj[j] = live ? sc[t * GQ + j] : -INFINITY;
+      float m = sj[j];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) red[warp * GQ + j] = m;
+    }
+    __syncthreads();
+    if (tid < GQ) {
+      float m = red[tid];
+      for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w * GQ + tid]);
+      stat[tid] = m;
+    }
+    __syncthreads();
+    float ls[GQ];
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+      const float pj = live ? __expf(sj[j] - stat[j]) : 0.0f;
+      ls[j] = pj;
+      const float ps = pj * kPScale;
+      const __half hi = __float2half_rn(ps);
+      const __half lo = __float2half_rn(ps - __half2float(hi));
+      pb[j * kChunk + t] = __half_as_ushort(hi);  // lo terms: column 4 + j (GQ <= 4) or 8 + j
+      pb[(NT == 2 ? 8 + j : 4 + j) * kChunk + t] = __half_as_ushort(lo);
+    }
+    if constexpr (NT == 1) {  // unused columns of the tile are zero
+      for (int j = GQ; j < 4; ++j) {
+        pb[j * kChunk + t] = 0;
+        pb[(4 + j) * kChunk + t] = 0;
+      }
+    }
+    __syncthreads();  // red is reused below
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+      float s16 = ls[j];  // per 16-token block (half a warp), then per warp
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) s16 += __shfl_xor_sync(0xffffffffu, s16, o);
+      if ((lane & 15) == 0) psum[(t >> 4) * GQ + j] = s16;
+      const float s32 = s16 + __shfl_xor_sync(0xffffffffu, s16, 16);
+      if (lane == 0) red[warp * GQ + j] = s32;
+    }
+  }
+  __syncthreads();
+
+  // ---- value sums on the tensor cores: warp w takes group w mod NG ----
+  // A = value codes transposed: row m = g is channel 2g of the group, m = g+8 is
+  // channel 2g+1; k slots 2c, 2c+1 / 2c+8, 2c+9 are tokens 4c, 4c+1 / 4c+2, 4c+3.
+  {
+    constexpr int WPG = 8 / NG;  // warps per group: 1 (d = 128) or 2 (d = 64)
+    const int r = warp % NG, part = warp / NG;
+    const int per = NBLK / WPG;
+    float o[NT][4];
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[tt][e] = 0.0f;
+    float oz[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // zero-point terms of this thread's (channel, head) pairs
+    for (int kb = part * per; kb < min(nblk, part * per + per); ++kb) {
+      const uint8_t* blk = vc + (kb * NG + r) * BLK;
+      uint32_t lo2[4], hi2[4];  // per token 4c + u: codes of channels 2g, 2g+1
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int bit = ((4 * c + u) * 16 + 2 * g) * BITS;
+        uint32_t v;
+        if constexpr (BITS == 4) {
+          v = blk[bit >> 3];
+        } else if constexpr (BITS == 8) {
+          v = *reinterpret_cast<const uint16_t*>(blk + (bit >> 3));
+        } else if constexpr (BITS == 2) {
+          v = (uint32_t)blk[bit >> 3] >> (bit & 7);
+        } else {
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(blk) + (bit >> 5);
+          v = __funnelshift_r(w[0], w[1], bit & 31);
+        }
+        constexpr uint32_t M = (1u << BITS) - 1u;
+        lo2[u] = v & M;
+        hi2[u] = (v >> BITS) & M;
+      }
+      uint32_t afr[4];
+      afr[0] = f16_sub1024(0x64006400u | lo2[0] | (lo2[1] << 16));
+      afr[1] = f16_sub1024(0x64006400u | hi2[0] | (hi2[1] << 16));
+      afr[2] = f16_sub1024(0x64006400u | lo2[2] | (lo2[3] << 16));
+      afr[3] = f16_sub1024(0x64006400u | hi2[2] | (hi2[3] << 16));
+      const float sv = vs[kb * NG + r] * (1.0f / kPScale), zv = vz[kb * NG + r];
+#pragma unroll
+      for (int tt = 0; tt < NT; ++tt) {
+        const uint2 bb = *reinterpret_cast<const uint2*>(pb + (tt * 8 + g) * kChunk + kb * 16 + 4 * c);
+        float d[4];
+        mma_f16_16816_z(d, afr, bb.x, bb.y);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[tt][e] = __fmaf_rn(sv, d[e], o[tt][e]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 2 * c + (e & 1);
+        if (j < GQ) oz[e] = __fmaf_rn(zv, psum[kb * GQ + j], oz[e]);
+      }
+    }
+    float ov[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (NT == 2) {
+        ov[e] = o[0][e] + o[1][e];
+      } else {
+        ov[e] = o[0][e] + __shfl_xor_sync(0xffffffffu, o[0][e], 2);
+      }
+      ov[e] += oz[e];
+    }
+    // d[e]: channel 2g + (e >> 1) of group r, head 2c + (e & 1)
+    float* out = a.partial + ((((long long)lz * a.k.B + b) * a.hq + h * GQ) * a.n_chunks + chunk) * (D + 2);
+    const long long head_stride = (long long)a.n_chunks * (D + 2);
+    const bool mine = NT == 2 || c < 2;
+    if constexpr (WPG == 1) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 2 * c + (e & 1);
+        if (mine && j < GQ) out[j * head_stride + 2 + 16 * r + 2 * g + (e >> 1)] = ov[e];
+      }
+    } else {  // two warps per group: add the halves in a fixed order through shared memory
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 2 * c + (e & 1);
+        if (mine && j < GQ) po[(part * GQ + j) * D + 16 * r + 2 * g + (e >> 1)] = ov[e];
+      }
+      __syncthreads();
+      for (int e = tid; e < GQ * D; e += kAttnThreads) {
+        const int j = e / D, cc = e % D;
+        out[j * head_stride + 2 + cc] = po[j * D + cc] + po[(GQ + j) * D + cc];
+      }
+    }
+    if (tid < GQ) {
+      float s = 0.0f;
+      for (int w = 0; w < 8; ++w) s += red[w * GQ + tid];
+      out[tid * head_stride + 0] = stat[tid];
+      out[tid * head_stride + 1] = s;
+    }
   }
 }
 
@@ -293,9 +405,9 @@ cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {
   constexpr int NG = D / 16;
   constexpr int CODE_BYTES = kChunk * D * BITS / 8;
   constexpr int NBLK = kChunk / 16;
-  static_assert((kAttnThreads / D) * GQ * D == kChunk * GQ, "the value parts' sums fit where the weights were");
-  const int smem_floats = 4 * NBLK * NG + GQ * D + GQ * NG + kChunk * GQ + 8 * GQ + GQ;
-  const size_t smem = 2 * CODE_BYTES + 16 + 4 * (size_t)smem_floats;
+  constexpr int NCOL = GQ == 8 ? 16 : 8;
+  const int smem_floats = 4 * NBLK * NG + GQ * D + GQ * NG + 8 + kChunk * GQ + NBLK * GQ + 8 * GQ + 8 + 2 * GQ * D;
+  const size_t smem = 2 * (CODE_BYTES + 16) + 4 * (size_t)smem_floats + 2 * (size_t)NCOL * kChunk;
   auto kern = attn_partial_kernel<D, BITS, GQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

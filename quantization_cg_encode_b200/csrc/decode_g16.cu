@@ -30,24 +30,6 @@ namespace cg {
 
 namespace {
 
-
-
-__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// fp16 pair {c_lo, c_hi} of two codes (< 256): the fp16 bit patterns
-// 0x6400 | c are exactly 1024 + c, and one exact f16x2 subtraction removes the
-// 1024.  No conversion instruction is involved.
-__device__ __forceinline__ uint32_t f16_sub1024(uint32_t biased) {
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(biased), "r"(0x64006400u));
-  return r;
-}
 __device__ __forceinline__ uint32_t f16pair(uint32_t c_lo, uint32_t c_hi) {
   return f16_sub1024(0x64006400u | c_lo | (c_hi << 16));
 }

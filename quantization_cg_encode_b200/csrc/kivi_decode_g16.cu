@@ -49,11 +49,6 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t f16_sub1024(uint32_t biased) {
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(biased), "r"(0x64006400u));
-  return r;
-}
 // fp16 pair {c_lo, c_hi} of two codes (< 256): 0x6400 | c is exactly 1024 + c
 __device__ __forceinline__ uint32_t f16pair(uint32_t c_lo, uint32_t c_hi) {
   return f16_sub1024(0x64006400u | c_lo | (c_hi << 16));
