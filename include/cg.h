@@ -65,9 +65,10 @@ typedef enum {
  * depend on the engine. */
 typedef enum {
   CG_ENGINE_AUTO = 0,         /* the fastest kernel for the request:
-                                 g = 16 with W = 16 (d 64 or 128): tensor-core
-                                 contraction with G split into two bf16 terms
-                                 (within about 2^-17 sum_j |G_ij x_j| of G x);
+                                 g = 16 with W = 16, and KIVI-style with g = 16
+                                 (d 64 or 128): tensor-core contraction with G
+                                 split into two bf16 terms (within about 2^-17
+                                 sum_j |G_ij x_j| of G x);
                                  g = d: tensor cores with G rounded to bf16;
                                  otherwise the fp32 FMA chain */
   CG_ENGINE_CUDA_CORES = 1,   /* the fp32 FMA chain on CUDA cores (g < d only):

@@ -193,7 +193,11 @@ cg_status cg_encode(const cg_kv_desc* kv, const cg_codec_desc* codec, const void
   a.gauged = gauged_dev;
   a.status = status_word();
   if (!a.status) return CG_ERR_CUDA;
-  if (a.kivi) return from_cuda(launch_kivi(a, true, num_sms(), (cudaStream_t)stream));
+  if (a.kivi) {
+    if (codec->engine == CG_ENGINE_AUTO && kivi_mma16_supported(a))
+      return from_cuda(launch_kivi_mma16(a, num_sms(), (cudaStream_t)stream));
+    return from_cuda(launch_kivi(a, true, num_sms(), (cudaStream_t)stream));
+  }
   if (a.g == kv->d_head) {
     if (kv->d_head != 128) return CG_ERR_UNSUPPORTED;
     return from_cuda(launch_fullhead(a, true, num_sms(), (cudaStream_t)stream));

@@ -32,6 +32,8 @@ bool codec_mma16_supported(const CodecArgs& a);
 cudaError_t launch_encode_mma16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_decode_mma16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_kivi(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);
+bool kivi_mma16_supported(const CodecArgs& a);
+cudaError_t launch_kivi_mma16(const CodecArgs& a, int num_sms, cudaStream_t st);
 bool kivi_decode_g16_supported(const CodecArgs& a);
 cudaError_t launch_kivi_decode_g16(const CodecArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_fullhead(const CodecArgs& a, bool encode, int num_sms, cudaStream_t st);

@@ -61,6 +61,24 @@ def oracle_quantize_own(y, bits, w):
     return dict(codes=oq.pack_codes(q, bits), z=z, s=s, q=q)
 
 
+def kivi_own_gauge(shape, codec):
+    """True when cg_encode's KIVI-style gauged values are its own two-term
+    tensor-core contraction (the default engine for g = 16, d_head 64 or 128)."""
+    return codec.mode == cg.KIVI and codec.g == 16 and shape[-1] in (64, 128) and codec.engine == cg.ENGINE_AUTO
+
+
+def oracle_kivi_own(y, bits):
+    """The oracle's KIVI-style quantizer (keys per channel over 32 tokens, values per
+    token over 32 channels) applied to the device's fp32 gauged values y
+    [L, 2, B, H, nt, d]: the layout of oracle.codec.encode_kivi's result."""
+    from oracle import quant as oq
+    y = np.asarray(y, np.float64)
+    qk, zk, sk = oq.quantize_ranges(oq.kivi_key_view(y[:, 0], 32), bits)
+    qv, zv, sv = oq.quantize_ranges(oq.kivi_value_view(y[:, 1], 32), bits)
+    return dict(key=dict(codes=oq.pack_codes(qk, bits), z=zk, s=sk, q=qk),
+                value=dict(codes=oq.pack_codes(qv, bits), z=zv, s=sv, q=qv), y=y)
+
+
 OWN_GAUGE_BOUND = 2.0 ** -16
 
 
