@@ -68,7 +68,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
   float* red = psum + NBLK * GQ;                 // [8 warps][GQ]
   float* stat = red + 8 * GQ;                    // [GQ]: chunk max
   float* po = stat + 8;                          // [2][GQ][D]: value halves (d = 64)
-  uint16_t* pb = reinterpret_cast<uint16_t*>(po + 2 * GQ * D);  // [NCOL][kChunk] fp16 p terms
+  float* zsum = po + 2 * GQ * D;                 // [NBLK][GQ]: sum_r z_r sum(q'_r) of each key block
+  uint32_t* bqs = reinterpret_cast<uint32_t*>(zsum + NBLK * GQ);  // [NG][NT][32 lanes][2] fp16 q'' fragments
+  uint16_t* pb = reinterpret_cast<uint16_t*>(bqs + NG * NT * 64);  // [NCOL][kChunk] fp16 p terms
 
   const int chunk = blockIdx.x;
   const int bh = blockIdx.y;  // b * H + h
@@ -131,30 +133,37 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
   }
   __syncthreads();
 
+  // Once per CTA: the B fragments of q'' (column n = g of tile tt holds q'' = q' 2^e
+  // of (term, head); k slots 2c, 2c+1 / 2c+8, 2c+9 are channels 4c, 4c+1 / 4c+2, 4c+3
+  // of the group), and the zero-point term of every (key block, head).
+  for (int e = tid; e < NG * NT * 32; e += kAttnThreads) {
+    const int ln = e & 31, tt = (e >> 5) % NT, r = (e >> 5) / NT;
+    const int gg = ln >> 2, cc = ln & 3;
+    const int j = NT == 2 ? gg : (gg & 3), lo = NT == 2 ? tt : (gg >> 2);
+    const bool on = j < GQ;
+    const float sj = on ? 1.0f / qinv[j] : 0.0f;
+    const float4 q4 = on ? *reinterpret_cast<const float4*>(qp + j * D + 16 * r + 4 * cc) : make_float4(0, 0, 0, 0);
+    const float v[4] = {q4.x * sj, q4.y * sj, q4.z * sj, q4.w * sj};
+    __half hv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __half hi = __float2half_rn(v[k]);
+      hv[k] = lo ? __float2half_rn(v[k] - __half2float(hi)) : hi;
+    }
+    bqs[2 * e] = (uint32_t)__half_as_ushort(hv[0]) | ((uint32_t)__half_as_ushort(hv[1]) << 16);
+    bqs[2 * e + 1] = (uint32_t)__half_as_ushort(hv[2]) | ((uint32_t)__half_as_ushort(hv[3]) << 16);
+  }
+  for (int e = tid; e < nblk * GQ; e += kAttnThreads) {
+    const int kb = e / GQ, j = e % GQ;
+    float zt = 0.0f;
+#pragma unroll
+    for (int r = 0; r < NG; ++r) zt = __fmaf_rn(kz[kb * NG + r], qsum[j * NG + r], zt);
+    zsum[e] = zt;
+  }
+  __syncthreads();
+
   // ---- scores on the tensor cores: warp w takes blocks w and w + 8 ----
   {
-    // B fragments: column n = g of tile tt holds q'' = q' 2^e of (term, head);
-    // k slots 2c, 2c+1 / 2c+8, 2c+9 are channels 4c, 4c+1 / 4c+2, 4c+3 of the group
-    uint32_t bq[NG][NT][2];
-#pragma unroll
-    for (int tt = 0; tt < NT; ++tt) {
-      const int j = NT == 2 ? g : (g & 3), lo = NT == 2 ? tt : (g >> 2);
-      const bool on = j < GQ;
-      const float sj = on ? 1.0f / qinv[j] : 0.0f;
-#pragma unroll
-      for (int r = 0; r < NG; ++r) {
-        float4 q4 = on ? *reinterpret_cast<const float4*>(qp + j * D + 16 * r + 4 * c) : make_float4(0, 0, 0, 0);
-        const float v[4] = {q4.x * sj, q4.y * sj, q4.z * sj, q4.w * sj};
-        __half hv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __half hi = __float2half_rn(v[e]);
-          hv[e] = lo ? __float2half_rn(v[e] - __half2float(hi)) : hi;
-        }
-        bq[r][tt][0] = (uint32_t)__half_as_ushort(hv[0]) | ((uint32_t)__half_as_ushort(hv[1]) << 16);
-        bq[r][tt][1] = (uint32_t)__half_as_ushort(hv[2]) | ((uint32_t)__half_as_ushort(hv[3]) << 16);
-      }
-    }
     const int bit_g = (16 * g + 4 * c) * BITS, bit_g8 = (16 * (g + 8) + 4 * c) * BITS;
 #pragma unroll
     for (int bi = 0; bi < 2; ++bi) {
@@ -195,8 +204,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
         const float sk = ks[kb * NG + r];
 #pragma unroll
         for (int tt = 0; tt < NT; ++tt) {
+          const uint2 bq = *reinterpret_cast<const uint2*>(bqs + 2 * ((r * NT + tt) * 32 + lane));
           float d[4];
-          mma_f16_16816_z(d, afr, bq[r][tt][0], bq[r][tt][1]);
+          mma_f16_16816_z(d, afr, bq.x, bq.y);
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[tt][e] = __fmaf_rn(sk, d[e], acc[tt][e]);
         }
@@ -214,12 +224,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int j = 2 * c + (e & 1), t = kb * 16 + g + 8 * (e >> 1);
-        if ((NT == 2 || c < 2) && j < GQ) {
-          float zt = 0.0f;
-#pragma unroll
-          for (int r = 0; r < NG; ++r) zt = __fmaf_rn(kz[kb * NG + r], qsum[j * NG + r], zt);
-          sc[t * GQ + j] = __fmaf_rn(sv[e], qinv[j], zt);
-        }
+        if ((NT == 2 || c < 2) && j < GQ) sc[t * GQ + j] = __fmaf_rn(sv[e], qinv[j], zsum[kb * GQ + j]);
       }
     }
   }
@@ -371,22 +376,44 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
 }
 
 // out[l][b][hq] = G_V^T (sum_k e^(m_k - M) o_k) / (sum_k e^(m_k - M) l_k)
+// (the chunk weights are formed once, in parallel, then every channel's sum
+// over the chunks reads independent partials)
 template <int D>
 __global__ void __launch_bounds__(D) attn_combine_kernel(AttnArgs a) {
-  constexpr int NG = D / 16;
+  constexpr int NG = D / 16, NW = D / 32;
+  extern __shared__ float wk[];  // [n_chunks] e^(m_k - M)
   __shared__ float og[D];
+  __shared__ float red[NW];
   const int hq = blockIdx.x, b = blockIdx.y, lz = blockIdx.z;
   const int l = a.l0 + lz, h = hq / (a.hq / a.k.H);
-  const int c = threadIdx.x;
+  const int c = threadIdx.x, lane = c & 31, w = c >> 5;
   const float* part = a.partial + ((((long long)lz * a.k.B + b) * a.hq + hq) * a.n_chunks) * (D + 2);
-  float M = -INFINITY;
-  for (int k = 0; k < a.n_chunks; ++k) M = fmaxf(M, part[k * (D + 2)]);
-  float Ls = 0.0f, O = 0.0f;
-  for (int k = 0; k < a.n_chunks; ++k) {
-    const float w = __expf(part[k * (D + 2)] - M);
-    Ls = __fmaf_rn(w, part[k * (D + 2) + 1], Ls);
-    O = __fmaf_rn(w, part[k * (D + 2) + 2 + c], O);
+  float m = -INFINITY;
+  for (int k = c; k < a.n_chunks; k += D) m = fmaxf(m, part[k * (D + 2)]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[w] = m;
+  __syncthreads();
+  float M = red[0];
+#pragma unroll
+  for (int i = 1; i < NW; ++i) M = fmaxf(M, red[i]);
+  float ls = 0.0f;
+  for (int k = c; k < a.n_chunks; k += D) {
+    const float wt = __expf(part[k * (D + 2)] - M);
+    wk[k] = wt;
+    ls = __fmaf_rn(wt, part[k * (D + 2) + 1], ls);
   }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+  __syncthreads();  // every thread has read red; the weights are in place
+  if (lane == 0) red[w] = ls;
+  __syncthreads();
+  float Ls = red[0];
+#pragma unroll
+  for (int i = 1; i < NW; ++i) Ls += red[i];
+  float O = 0.0f;
+#pragma unroll 4
+  for (int k = 0; k < a.n_chunks; ++k) O = __fmaf_rn(wk[k], part[k * (D + 2) + 2 + c], O);
   og[c] = O / Ls;
   __syncthreads();
   // x = G_V^T y per group: out[16 r + j] = sum_i G[r][i][j] y[16 r + i]
@@ -406,7 +433,9 @@ cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {
   constexpr int CODE_BYTES = kChunk * D * BITS / 8;
   constexpr int NBLK = kChunk / 16;
   constexpr int NCOL = GQ == 8 ? 16 : 8;
-  const int smem_floats = 4 * NBLK * NG + GQ * D + GQ * NG + 8 + kChunk * GQ + NBLK * GQ + 8 * GQ + 8 + 2 * GQ * D;
+  constexpr int NT = GQ == 8 ? 2 : 1;
+  const int smem_floats = 4 * NBLK * NG + GQ * D + GQ * NG + 8 + kChunk * GQ + NBLK * GQ + 8 * GQ + 8 + 2 * GQ * D +
+                          NBLK * GQ + NG * NT * 64;
   const size_t smem = 2 * (CODE_BYTES + 16) + 4 * (size_t)smem_floats + 2 * (size_t)NCOL * kChunk;
   auto kern = attn_partial_kernel<D, BITS, GQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -416,7 +445,12 @@ cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 cgrid(a.hq, a.k.B, a.n_layers);
-  attn_combine_kernel<D><<<cgrid, D, 0, st>>>(a);
+  const size_t csmem = (size_t)a.n_chunks * sizeof(float);
+  if (csmem > 48 * 1024) {
+    e = cudaFuncSetAttribute(attn_combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
+    if (e != cudaSuccess) return e;
+  }
+  attn_combine_kernel<D><<<cgrid, D, csmem, st>>>(a);
   return cudaGetLastError();
 }
 
