@@ -34,17 +34,36 @@ namespace cg {
 
 namespace {
 
-constexpr int kChunk = 256;  // tokens per CTA
+constexpr int kChunk = 256;  // tokens per chunk
+constexpr int kCpc = 4;      // chunks per CTA (one partial per CTA)
 constexpr int kAttnThreads = 256;
+
+// Asynchronous global -> shared copies (16 bytes bypassing L1, or 4 bytes),
+// grouped per thread; wait until at most N groups of this thread are pending.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 }  // namespace
 
-// partial[l][b][hq][chunk] = {m, l, o[D]} in gauge coordinates.
+// partial[l][b][hq][split] = {m, l, o[D]} in gauge coordinates, over the token
+// chunks [split kCpc, split kCpc + kCpc) of one (layer, batch, KV head).
 //
 // MMA columns: for GQ <= 4 one N = 8 tile holds the hi terms of heads 0..3 in
 // columns 0..3 and the lo terms in 4..7 (heads >= GQ are zero); for GQ = 8 a
 // tile of hi terms and a tile of lo terms.  A thread's accumulator columns 2c,
 // 2c+1 are then heads 2c, 2c+1 (hi) or their lo parts, combined by a shuffle.
+// A CTA's chunks stream through two shared-memory stages (cp.async: the next
+// chunk's codes, steps and zero points load while the current one computes)
+// and are merged with the online softmax rescaling.
 template <int D, int BITS, int GQ>
 __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) {
   constexpr int NG = D / 16;
@@ -52,57 +71,62 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
   constexpr int CODE_BYTES = kChunk * D * BITS / 8;
   constexpr int NBLK = kChunk / 16;
   constexpr int NT = GQ == 8 ? 2 : 1;            // N = 8 tiles per MMA step
+  constexpr int RB = NBLK * NG * 2;              // bytes of one chunk's fp16 steps (or zero points)
+  constexpr int STAGE = 2 * (CODE_BYTES + 16) + 4 * RB;
   constexpr float kPScale = 4096.0f;             // p in [0, 1] -> [0, 2^12] for fp16 terms
   extern __shared__ __align__(16) unsigned char smem[];
-  uint8_t* kc = smem;                            // key codes of the chunk
-  uint8_t* vc = kc + CODE_BYTES + 16;            // value codes (16 B slack after each)
-  float* ks = reinterpret_cast<float*>(vc + CODE_BYTES + 16);  // [NBLK][NG] key steps
-  float* kz = ks + NBLK * NG;
-  float* vs = kz + NBLK * NG;
-  float* vz = vs + NBLK * NG;
-  float* qp = vz + NBLK * NG;                    // [GQ][D]: q' = scale * G_K q
+  // stage b: [key codes | 16 | value codes | 16 | key steps | key zeros | value steps | value zeros]
+  float* qp = reinterpret_cast<float*>(smem + 2 * STAGE);  // [GQ][D]: q' = scale * G_K q
   float* qsum = qp + GQ * D;                     // [GQ][NG]: sum of q' over each group
   float* qinv = qsum + GQ * NG;                  // [GQ]: 2^-e_j, the inverse of q''s fp16 scaling
   float* sc = qinv + 8;                          // [kChunk][GQ]: scores
   float* psum = sc + kChunk * GQ;                // [NBLK][GQ]: sum of p over each block
   float* red = psum + NBLK * GQ;                 // [8 warps][GQ]
   float* stat = red + 8 * GQ;                    // [GQ]: chunk max
-  float* po = stat + 8;                          // [2][GQ][D]: value halves (d = 64)
+  float* run = stat + 8;                         // [4][8]: running max, running sum, old / new weights
+  float* po = run + 32;                          // [2][GQ][D]: value halves (d = 64)
   float* zsum = po + 2 * GQ * D;                 // [NBLK][GQ]: sum_r z_r sum(q'_r) of each key block
   uint32_t* bqs = reinterpret_cast<uint32_t*>(zsum + NBLK * GQ);  // [NG][NT][32 lanes][2] fp16 q'' fragments
   uint16_t* pb = reinterpret_cast<uint16_t*>(bqs + NG * NT * 64);  // [NCOL][kChunk] fp16 p terms
 
-  const int chunk = blockIdx.x;
+  const int split = blockIdx.x;
   const int bh = blockIdx.y;  // b * H + h
   const int lz = blockIdx.z;  // layer index within the call
   const int l = a.l0 + lz;
   const int h = bh % a.k.H, b = bh / a.k.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int t0 = chunk * kChunk;
-  const int ntok = min(kChunk, a.n_tokens - t0);
-  const int nblk = ntok / 16;  // n_tokens is a multiple of 16
+  const int n_tc = (a.n_tokens + kChunk - 1) / kChunk;  // token chunks
+  const int c0 = split * kCpc, c1 = min(n_tc, c0 + kCpc);
   const long long slice_k = (((long long)l * 2 + 0) * a.k.B + b) * a.k.H + h;
   const long long slice_v = (((long long)l * 2 + 1) * a.k.B + b) * a.k.H + h;
   const long long slice_bytes = (long long)a.k.T * D * BITS / 8;
   const int T16 = a.k.T / 16;
 
-  // stage codes (whole range blocks), steps and zero points; q' per group
-  {
-    const uint4* srck = reinterpret_cast<const uint4*>(a.codes + slice_k * slice_bytes + (long long)(t0 / 16) * NG * BLK);
-    const uint4* srcv = reinterpret_cast<const uint4*>(a.codes + slice_v * slice_bytes + (long long)(t0 / 16) * NG * BLK);
-    const int n16 = nblk * NG * BLK / 16;
+  // chunk -> stage st: 16-byte copies of the codes, 4-byte copies of the ranges
+  auto issue = [&](int chunk, int st) {
+    unsigned char* base = smem + st * STAGE;
+    const int t0 = chunk * kChunk, nb = min(kChunk, a.n_tokens - t0) / 16;
+    const uint8_t* srck = a.codes + slice_k * slice_bytes + (long long)(t0 / 16) * NG * BLK;
+    const uint8_t* srcv = a.codes + slice_v * slice_bytes + (long long)(t0 / 16) * NG * BLK;
+    const int n16 = nb * NG * BLK / 16;
     for (int e = tid; e < n16; e += kAttnThreads) {
-      reinterpret_cast<uint4*>(kc)[e] = __ldg(srck + e);
-      reinterpret_cast<uint4*>(vc)[e] = __ldg(srcv + e);
+      cp_async16(base + 16 * e, srck + 16 * e);
+      cp_async16(base + CODE_BYTES + 16 + 16 * e, srcv + 16 * e);
     }
-    for (int e = tid; e < nblk * NG; e += kAttnThreads) {
-      const long long ik = (slice_k * T16 + t0 / 16) * NG + e, iv = (slice_v * T16 + t0 / 16) * NG + e;
-      ks[e] = __half2float(__ushort_as_half(a.scales[ik]));
-      kz[e] = __half2float(__ushort_as_half(a.zeros[ik]));
-      vs[e] = __half2float(__ushort_as_half(a.scales[iv]));
-      vz[e] = __half2float(__ushort_as_half(a.zeros[iv]));
+    const int n4 = nb * NG / 2;  // 4-byte words of one range array
+    for (int e = tid; e < 4 * n4; e += kAttnThreads) {
+      const int arr = e / n4, w = e % n4;  // key steps, key zeros, value steps, value zeros
+      const uint16_t* src = (arr & 1) ? a.zeros : a.scales;
+      const long long sl = (arr >> 1) ? slice_v : slice_k;
+      cp_async4(base + 2 * (CODE_BYTES + 16) + arr * RB + 4 * w, src + (sl * T16 + t0 / 16) * NG + 2 * w);
     }
+    cp_async_commit();
+  };
+  issue(c0, 0);  // the first chunk loads while q' is formed
+
+  // q' per group, once per CTA
+  {
     const float* Gk = a.G + gauge_set(l, 0, h, a.k) * NG * 256;
     for (int e = tid; e < GQ * D; e += kAttnThreads) {
       const int j = e / D, cc = e % D, r = cc >> 4, i = cc & 15;
@@ -112,6 +136,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
 #pragma unroll
       for (int m = 0; m < 16; ++m) acc = __fmaf_rn(gi[m], bf16lo((uint32_t)qrow[m]), acc);
       qp[e] = acc * a.scale;
+    }
+    if (tid < GQ) {
+      run[tid] = -INFINITY;  // running max
+      run[8 + tid] = 0.0f;   // running sum
     }
   }
   __syncthreads();
@@ -132,10 +160,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
     if (lane == 0) qinv[warp] = m > 0.0f ? ldexpf(1.0f, ex - 15) : 1.0f;
   }
   __syncthreads();
-
-  // Once per CTA: the B fragments of q'' (column n = g of tile tt holds q'' = q' 2^e
-  // of (term, head); k slots 2c, 2c+1 / 2c+8, 2c+9 are channels 4c, 4c+1 / 4c+2, 4c+3
-  // of the group), and the zero-point term of every (key block, head).
+  // the B fragments of q'' (column n = g of tile tt holds q'' = q' 2^e of (term,
+  // head); k slots 2c, 2c+1 / 2c+8, 2c+9 are channels 4c, 4c+1 / 4c+2, 4c+3 of the group)
   for (int e = tid; e < NG * NT * 32; e += kAttnThreads) {
     const int ln = e & 31, tt = (e >> 5) % NT, r = (e >> 5) / NT;
     const int gg = ln >> 2, cc = ln & 3;
@@ -153,224 +179,268 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
     bqs[2 * e] = (uint32_t)__half_as_ushort(hv[0]) | ((uint32_t)__half_as_ushort(hv[1]) << 16);
     bqs[2 * e + 1] = (uint32_t)__half_as_ushort(hv[2]) | ((uint32_t)__half_as_ushort(hv[3]) << 16);
   }
-  for (int e = tid; e < nblk * GQ; e += kAttnThreads) {
-    const int kb = e / GQ, j = e % GQ;
-    float zt = 0.0f;
-#pragma unroll
-    for (int r = 0; r < NG; ++r) zt = __fmaf_rn(kz[kb * NG + r], qsum[j * NG + r], zt);
-    zsum[e] = zt;
-  }
-  __syncthreads();
 
-  // ---- scores on the tensor cores: warp w takes blocks w and w + 8 ----
-  {
-    const int bit_g = (16 * g + 4 * c) * BITS, bit_g8 = (16 * (g + 8) + 4 * c) * BITS;
-#pragma unroll
-    for (int bi = 0; bi < 2; ++bi) {
-      const int kb = warp + 8 * bi;
-      if (kb >= nblk) continue;  // warp-uniform
-      float acc[NT][4];
-#pragma unroll
-      for (int tt = 0; tt < NT; ++tt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[tt][e] = 0.0f;
-#pragma unroll
-      for (int r = 0; r < NG; ++r) {
-        const uint8_t* blk = kc + (kb * NG + r) * BLK;
-        uint32_t cv[2];  // rows g, g+8: codes 4c .. 4c+3 (4 BITS bits, low aligned)
-        if constexpr (BITS == 4) {
-          cv[0] = *reinterpret_cast<const uint16_t*>(blk + (bit_g >> 3));
-          cv[1] = *reinterpret_cast<const uint16_t*>(blk + (bit_g8 >> 3));
-        } else if constexpr (BITS == 8) {
-          cv[0] = *reinterpret_cast<const uint32_t*>(blk + (bit_g >> 3));
-          cv[1] = *reinterpret_cast<const uint32_t*>(blk + (bit_g8 >> 3));
-        } else if constexpr (BITS == 2) {
-          cv[0] = blk[bit_g >> 3];
-          cv[1] = blk[bit_g8 >> 3];
-        } else {
-          const uint32_t* w0 = reinterpret_cast<const uint32_t*>(blk) + (bit_g >> 5);
-          const uint32_t* w1 = reinterpret_cast<const uint32_t*>(blk) + (bit_g8 >> 5);
-          cv[0] = __funnelshift_r(w0[0], w0[1], bit_g & 31);
-          cv[1] = __funnelshift_r(w1[0], w1[1], bit_g8 & 31);
-        }
-        uint32_t afr[4];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          constexpr uint32_t M = (1u << BITS) - 1u;
-          const uint32_t v = cv[hh];
-          afr[hh] = f16_sub1024(0x64006400u | (v & M) | (((v >> BITS) & M) << 16));
-          afr[2 + hh] = f16_sub1024(0x64006400u | ((v >> (2 * BITS)) & M) | (((v >> (3 * BITS)) & M) << 16));
-        }
-        const float sk = ks[kb * NG + r];
-#pragma unroll
-        for (int tt = 0; tt < NT; ++tt) {
-          const uint2 bq = *reinterpret_cast<const uint2*>(bqs + 2 * ((r * NT + tt) * 32 + lane));
-          float d[4];
-          mma_f16_16816_z(d, afr, bq.x, bq.y);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[tt][e] = __fmaf_rn(sk, d[e], acc[tt][e]);
-        }
-      }
-      // hi + lo terms; then columns 2c, 2c+1 are heads 2c, 2c+1 (threads c < 2 for GQ <= 4)
-      float sv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if constexpr (NT == 2) {
-          sv[e] = acc[0][e] + acc[1][e];
-        } else {
-          sv[e] = acc[0][e] + __shfl_xor_sync(0xffffffffu, acc[0][e], 2);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = 2 * c + (e & 1), t = kb * 16 + g + 8 * (e >> 1);
-        if ((NT == 2 || c < 2) && j < GQ) sc[t * GQ + j] = __fmaf_rn(sv[e], qinv[j], zsum[kb * GQ + j]);
-      }
+  float orun[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // running o of this thread's (channel, head) pairs
+  for (int chunk = c0, it = 0; chunk < c1; ++chunk, ++it) {
+    const int st = it & 1;
+    __syncthreads();  // every thread is done with the other stage (the previous chunk)
+    if (chunk + 1 < c1) {
+      issue(chunk + 1, st ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-  }
-  __syncthreads();
-
-  // ---- softmax over the chunk, thread = token ----
-  {
-    const int t = tid;
-    const bool live = t < ntok;
-    float sj[GQ];
+    __syncthreads();  // this chunk's stage is complete
+    const unsigned char* base = smem + st * STAGE;
+    const uint8_t* kc = base;
+    const uint8_t* vc = base + CODE_BYTES + 16;
+    const __half* ks = reinterpret_cast<const __half*>(base + 2 * (CODE_BYTES + 16));
+    const __half* kz = ks + RB / 2;
+    const __half* vs = kz + RB / 2;
+    const __half* vz = vs + RB / 2;
+    const int t0 = chunk * kChunk;
+    const int ntok = min(kChunk, a.n_tokens - t0);
+    const int nblk = ntok / 16;  // n_tokens is a multiple of 16
+    for (int e = tid; e < nblk * GQ; e += kAttnThreads) {
+      const int kb = e / GQ, j = e % GQ;
+      float zt = 0.0f;
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-      sj[j] = live ? sc[t * GQ + j] : -INFINITY;
-      float m = sj[j];
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == 0) red[warp * GQ + j] = m;
+      for (int r = 0; r < NG; ++r) zt = __fmaf_rn(__half2float(kz[kb * NG + r]), qsum[j * NG + r], zt);
+      zsum[e] = zt;
     }
     __syncthreads();
-    if (tid < GQ) {
-      float m = red[tid];
-      for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w * GQ + tid]);
-      stat[tid] = m;
+
+    // ---- scores on the tensor cores: warp w takes blocks w and w + 8 ----
+    {
+      const int bit_g = (16 * g + 4 * c) * BITS, bit_g8 = (16 * (g + 8) + 4 * c) * BITS;
+  #pragma unroll
+      for (int bi = 0; bi < 2; ++bi) {
+        const int kb = warp + 8 * bi;
+        if (kb >= nblk) continue;  // warp-uniform
+        float acc[NT][4];
+  #pragma unroll
+        for (int tt = 0; tt < NT; ++tt)
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) acc[tt][e] = 0.0f;
+  #pragma unroll
+        for (int r = 0; r < NG; ++r) {
+          const uint8_t* blk = kc + (kb * NG + r) * BLK;
+          uint32_t cv[2];  // rows g, g+8: codes 4c .. 4c+3 (4 BITS bits, low aligned)
+          if constexpr (BITS == 4) {
+            cv[0] = *reinterpret_cast<const uint16_t*>(blk + (bit_g >> 3));
+            cv[1] = *reinterpret_cast<const uint16_t*>(blk + (bit_g8 >> 3));
+          } else if constexpr (BITS == 8) {
+            cv[0] = *reinterpret_cast<const uint32_t*>(blk + (bit_g >> 3));
+            cv[1] = *reinterpret_cast<const uint32_t*>(blk + (bit_g8 >> 3));
+          } else if constexpr (BITS == 2) {
+            cv[0] = blk[bit_g >> 3];
+            cv[1] = blk[bit_g8 >> 3];
+          } else {
+            const uint32_t* w0 = reinterpret_cast<const uint32_t*>(blk) + (bit_g >> 5);
+            const uint32_t* w1 = reinterpret_cast<const uint32_t*>(blk) + (bit_g8 >> 5);
+            cv[0] = __funnelshift_r(w0[0], w0[1], bit_g & 31);
+            cv[1] = __funnelshift_r(w1[0], w1[1], bit_g8 & 31);
+          }
+          uint32_t afr[4];
+  #pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            constexpr uint32_t M = (1u << BITS) - 1u;
+            const uint32_t v = cv[hh];
+            afr[hh] = f16_sub1024(0x64006400u | (v & M) | (((v >> BITS) & M) << 16));
+            afr[2 + hh] = f16_sub1024(0x64006400u | ((v >> (2 * BITS)) & M) | (((v >> (3 * BITS)) & M) << 16));
+          }
+          const float sk = __half2float(ks[kb * NG + r]);
+  #pragma unroll
+          for (int tt = 0; tt < NT; ++tt) {
+            const uint2 bq = *reinterpret_cast<const uint2*>(bqs + 2 * ((r * NT + tt) * 32 + lane));
+            float d[4];
+            mma_f16_16816_z(d, afr, bq.x, bq.y);
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) acc[tt][e] = __fmaf_rn(sk, d[e], acc[tt][e]);
+          }
+        }
+        // hi + lo terms; then columns 2c, 2c+1 are heads 2c, 2c+1 (threads c < 2 for GQ <= 4)
+        float sv[4];
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (NT == 2) {
+            sv[e] = acc[0][e] + acc[1][e];
+          } else {
+            sv[e] = acc[0][e] + __shfl_xor_sync(0xffffffffu, acc[0][e], 2);
+          }
+        }
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 2 * c + (e & 1), t = kb * 16 + g + 8 * (e >> 1);
+          if ((NT == 2 || c < 2) && j < GQ) sc[t * GQ + j] = __fmaf_rn(sv[e], qinv[j], zsum[kb * GQ + j]);
+        }
+      }
     }
     __syncthreads();
-    float ls[GQ];
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-      const float pj = live ? __expf(sj[j] - stat[j]) : 0.0f;
-      ls[j] = pj;
-      const float ps = pj * kPScale;
-      const __half hi = __float2half_rn(ps);
-      const __half lo = __float2half_rn(ps - __half2float(hi));
-      pb[j * kChunk + t] = __half_as_ushort(hi);  // lo terms: column 4 + j (GQ <= 4) or 8 + j
-      pb[(NT == 2 ? 8 + j : 4 + j) * kChunk + t] = __half_as_ushort(lo);
-    }
-    if constexpr (NT == 1) {  // unused columns of the tile are zero
-      for (int j = GQ; j < 4; ++j) {
-        pb[j * kChunk + t] = 0;
-        pb[(4 + j) * kChunk + t] = 0;
-      }
-    }
-    __syncthreads();  // red is reused below
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-      float s16 = ls[j];  // per 16-token block (half a warp), then per warp
-#pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) s16 += __shfl_xor_sync(0xffffffffu, s16, o);
-      if ((lane & 15) == 0) psum[(t >> 4) * GQ + j] = s16;
-      const float s32 = s16 + __shfl_xor_sync(0xffffffffu, s16, 16);
-      if (lane == 0) red[warp * GQ + j] = s32;
-    }
-  }
-  __syncthreads();
 
-  // ---- value sums on the tensor cores: warp w takes group w mod NG ----
-  // A = value codes transposed: row m = g is channel 2g of the group, m = g+8 is
-  // channel 2g+1; k slots 2c, 2c+1 / 2c+8, 2c+9 are tokens 4c, 4c+1 / 4c+2, 4c+3.
-  {
-    constexpr int WPG = 8 / NG;  // warps per group: 1 (d = 128) or 2 (d = 64)
-    const int r = warp % NG, part = warp / NG;
-    const int per = NBLK / WPG;
-    float o[NT][4];
-#pragma unroll
-    for (int tt = 0; tt < NT; ++tt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[tt][e] = 0.0f;
-    float oz[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // zero-point terms of this thread's (channel, head) pairs
-    for (int kb = part * per; kb < min(nblk, part * per + per); ++kb) {
-      const uint8_t* blk = vc + (kb * NG + r) * BLK;
-      uint32_t lo2[4], hi2[4];  // per token 4c + u: codes of channels 2g, 2g+1
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int bit = ((4 * c + u) * 16 + 2 * g) * BITS;
-        uint32_t v;
-        if constexpr (BITS == 4) {
-          v = blk[bit >> 3];
-        } else if constexpr (BITS == 8) {
-          v = *reinterpret_cast<const uint16_t*>(blk + (bit >> 3));
-        } else if constexpr (BITS == 2) {
-          v = (uint32_t)blk[bit >> 3] >> (bit & 7);
-        } else {
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(blk) + (bit >> 5);
-          v = __funnelshift_r(w[0], w[1], bit & 31);
-        }
-        constexpr uint32_t M = (1u << BITS) - 1u;
-        lo2[u] = v & M;
-        hi2[u] = (v >> BITS) & M;
-      }
-      uint32_t afr[4];
-      afr[0] = f16_sub1024(0x64006400u | lo2[0] | (lo2[1] << 16));
-      afr[1] = f16_sub1024(0x64006400u | hi2[0] | (hi2[1] << 16));
-      afr[2] = f16_sub1024(0x64006400u | lo2[2] | (lo2[3] << 16));
-      afr[3] = f16_sub1024(0x64006400u | hi2[2] | (hi2[3] << 16));
-      const float sv = vs[kb * NG + r] * (1.0f / kPScale), zv = vz[kb * NG + r];
-#pragma unroll
-      for (int tt = 0; tt < NT; ++tt) {
-        const uint2 bb = *reinterpret_cast<const uint2*>(pb + (tt * 8 + g) * kChunk + kb * 16 + 4 * c);
-        float d[4];
-        mma_f16_16816_z(d, afr, bb.x, bb.y);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[tt][e] = __fmaf_rn(sv, d[e], o[tt][e]);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = 2 * c + (e & 1);
-        if (j < GQ) oz[e] = __fmaf_rn(zv, psum[kb * GQ + j], oz[e]);
-      }
-    }
-    float ov[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if constexpr (NT == 2) {
-        ov[e] = o[0][e] + o[1][e];
-      } else {
-        ov[e] = o[0][e] + __shfl_xor_sync(0xffffffffu, o[0][e], 2);
-      }
-      ov[e] += oz[e];
-    }
-    // d[e]: channel 2g + (e >> 1) of group r, head 2c + (e & 1)
-    float* out = a.partial + ((((long long)lz * a.k.B + b) * a.hq + h * GQ) * a.n_chunks + chunk) * (D + 2);
-    const long long head_stride = (long long)a.n_chunks * (D + 2);
-    const bool mine = NT == 2 || c < 2;
-    if constexpr (WPG == 1) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = 2 * c + (e & 1);
-        if (mine && j < GQ) out[j * head_stride + 2 + 16 * r + 2 * g + (e >> 1)] = ov[e];
-      }
-    } else {  // two warps per group: add the halves in a fixed order through shared memory
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = 2 * c + (e & 1);
-        if (mine && j < GQ) po[(part * GQ + j) * D + 16 * r + 2 * g + (e >> 1)] = ov[e];
+    // ---- softmax over the chunk, thread = token ----
+    {
+      const int t = tid;
+      const bool live = t < ntok;
+      float sj[GQ];
+  #pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        sj[j] = live ? sc[t * GQ + j] : -INFINITY;
+        float m = sj[j];
+  #pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) red[warp * GQ + j] = m;
       }
       __syncthreads();
-      for (int e = tid; e < GQ * D; e += kAttnThreads) {
-        const int j = e / D, cc = e % D;
-        out[j * head_stride + 2 + cc] = po[j * D + cc] + po[(GQ + j) * D + cc];
+      if (tid < GQ) {
+        float m = red[tid];
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w * GQ + tid]);
+        stat[tid] = m;
+      }
+      __syncthreads();
+      float ls[GQ];
+  #pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        const float pj = live ? __expf(sj[j] - stat[j]) : 0.0f;
+        ls[j] = pj;
+        const float ps = pj * kPScale;
+        const __half hi = __float2half_rn(ps);
+        const __half lo = __float2half_rn(ps - __half2float(hi));
+        pb[j * kChunk + t] = __half_as_ushort(hi);  // lo terms: column 4 + j (GQ <= 4) or 8 + j
+        pb[(NT == 2 ? 8 + j : 4 + j) * kChunk + t] = __half_as_ushort(lo);
+      }
+      if constexpr (NT == 1) {  // unused columns of the tile are zero
+        for (int j = GQ; j < 4; ++j) {
+          pb[j * kChunk + t] = 0;
+          pb[(4 + j) * kChunk + t] = 0;
+        }
+      }
+      __syncthreads();  // red is reused below
+  #pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        float s16 = ls[j];  // per 16-token block (half a warp), then per warp
+  #pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) s16 += __shfl_xor_sync(0xffffffffu, s16, o);
+        if ((lane & 15) == 0) psum[(t >> 4) * GQ + j] = s16;
+        const float s32 = s16 + __shfl_xor_sync(0xffffffffu, s16, 16);
+        if (lane == 0) red[warp * GQ + j] = s32;
       }
     }
+    __syncthreads();
+
+    // ---- value sums on the tensor cores: warp w takes group w mod NG ----
+    // A = value codes transposed: row m = g is channel 2g of the group, m = g+8 is
+    // channel 2g+1; k slots 2c, 2c+1 / 2c+8, 2c+9 are tokens 4c, 4c+1 / 4c+2, 4c+3.
+    {
+      constexpr int WPG = 8 / NG;  // warps per group: 1 (d = 128) or 2 (d = 64)
+      const int r = warp % NG, part = warp / NG;
+      const int per = NBLK / WPG;
+      float o[NT][4];
+  #pragma unroll
+      for (int tt = 0; tt < NT; ++tt)
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) o[tt][e] = 0.0f;
+      float oz[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // zero-point terms of this thread's (channel, head) pairs
+      for (int kb = part * per; kb < min(nblk, part * per + per); ++kb) {
+        const uint8_t* blk = vc + (kb * NG + r) * BLK;
+        uint32_t lo2[4], hi2[4];  // per token 4c + u: codes of channels 2g, 2g+1
+  #pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int bit = ((4 * c + u) * 16 + 2 * g) * BITS;
+          uint32_t v;
+          if constexpr (BITS == 4) {
+            v = blk[bit >> 3];
+          } else if constexpr (BITS == 8) {
+            v = *reinterpret_cast<const uint16_t*>(blk + (bit >> 3));
+          } else if constexpr (BITS == 2) {
+            v = (uint32_t)blk[bit >> 3] >> (bit & 7);
+          } else {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(blk) + (bit >> 5);
+            v = __funnelshift_r(w[0], w[1], bit & 31);
+          }
+          constexpr uint32_t M = (1u << BITS) - 1u;
+          lo2[u] = v & M;
+          hi2[u] = (v >> BITS) & M;
+        }
+        uint32_t afr[4];
+        afr[0] = f16_sub1024(0x64006400u | lo2[0] | (lo2[1] << 16));
+        afr[1] = f16_sub1024(0x64006400u | hi2[0] | (hi2[1] << 16));
+        afr[2] = f16_sub1024(0x64006400u | lo2[2] | (lo2[3] << 16));
+        afr[3] = f16_sub1024(0x64006400u | hi2[2] | (hi2[3] << 16));
+        const float sv = __half2float(vs[kb * NG + r]) * (1.0f / kPScale), zv = __half2float(vz[kb * NG + r]);
+  #pragma unroll
+        for (int tt = 0; tt < NT; ++tt) {
+          const uint2 bb = *reinterpret_cast<const uint2*>(pb + (tt * 8 + g) * kChunk + kb * 16 + 4 * c);
+          float d[4];
+          mma_f16_16816_z(d, afr, bb.x, bb.y);
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) o[tt][e] = __fmaf_rn(sv, d[e], o[tt][e]);
+        }
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 2 * c + (e & 1);
+          if (j < GQ) oz[e] = __fmaf_rn(zv, psum[kb * GQ + j], oz[e]);
+        }
+      }
+      float ov[4];
+  #pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if constexpr (NT == 2) {
+          ov[e] = o[0][e] + o[1][e];
+        } else {
+          ov[e] = o[0][e] + __shfl_xor_sync(0xffffffffu, o[0][e], 2);
+        }
+        ov[e] += oz[e];
+      }
+    // ov[e]: channel 2g + (e >> 1) of group r, head 2c + (e & 1) (d = 64: the halves added in order)
+      const bool mine = (NT == 2 || c < 2) && part == 0;
+      if constexpr (WPG == 2) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 2 * c + (e & 1);
+          if ((NT == 2 || c < 2) && j < GQ) po[(part * GQ + j) * D + 16 * r + 2 * g + (e >> 1)] = ov[e];
+        }
+      }
+      // online softmax: merge this chunk into the running (max, sum, o)
+      if (tid < GQ) {
+        float s = 0.0f;
+        for (int w = 0; w < 8; ++w) s += red[w * GQ + tid];
+        const float m_old = run[tid], m_new = fmaxf(m_old, stat[tid]);
+        const float w_old = __expf(m_old - m_new), w_new = __expf(stat[tid] - m_new);
+        run[tid] = m_new;
+        run[8 + tid] = __fmaf_rn(run[8 + tid], w_old, s * w_new);
+        run[16 + tid] = w_old;
+        run[24 + tid] = w_new;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 2 * c + (e & 1);
+        if (mine && j < GQ) {
+          float v = ov[e];
+          if constexpr (WPG == 2) {
+            const int ch = 16 * r + 2 * g + (e >> 1);
+            v = po[j * D + ch] + po[(GQ + j) * D + ch];
+          }
+          orun[e] = __fmaf_rn(orun[e], run[16 + j], v * run[24 + j]);
+        }
+      }
+    }
+  }
+  // write this split's partial
+  {
+    const int r = warp % NG, part = warp / NG;
+    float* out = a.partial + ((((long long)lz * a.k.B + b) * a.hq + h * GQ) * a.n_chunks + split) * (D + 2);
+    const long long head_stride = (long long)a.n_chunks * (D + 2);
+    const bool mine = (NT == 2 || c < 2) && part == 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 2 * c + (e & 1);
+      if (mine && j < GQ) out[j * head_stride + 2 + 16 * r + 2 * g + (e >> 1)] = orun[e];
+    }
     if (tid < GQ) {
-      float s = 0.0f;
-      for (int w = 0; w < 8; ++w) s += red[w * GQ + tid];
-      out[tid * head_stride + 0] = stat[tid];
-      out[tid * head_stride + 1] = s;
+      out[tid * head_stride + 0] = run[tid];
+      out[tid * head_stride + 1] = run[8 + tid];
     }
   }
 }
@@ -432,15 +502,16 @@ cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {
   constexpr int NG = D / 16;
   constexpr int CODE_BYTES = kChunk * D * BITS / 8;
   constexpr int NBLK = kChunk / 16;
-  constexpr int NCOL = GQ == 8 ? 16 : 8;
   constexpr int NT = GQ == 8 ? 2 : 1;
-  const int smem_floats = 4 * NBLK * NG + GQ * D + GQ * NG + 8 + kChunk * GQ + NBLK * GQ + 8 * GQ + 8 + 2 * GQ * D +
-                          NBLK * GQ + NG * NT * 64;
-  const size_t smem = 2 * (CODE_BYTES + 16) + 4 * (size_t)smem_floats + 2 * (size_t)NCOL * kChunk;
+  constexpr int NCOL = 8 * NT;
+  constexpr int STAGE = 2 * (CODE_BYTES + 16) + 4 * NBLK * NG * 2;
+  const int smem_floats = GQ * D + GQ * NG + 8 + kChunk * GQ + NBLK * GQ + 8 * GQ + 8 + 32 + 2 * GQ * D + NBLK * GQ +
+                          NG * NT * 64;
+  const size_t smem = 2 * (size_t)STAGE + 4 * (size_t)smem_floats + 2 * (size_t)NCOL * kChunk;
   auto kern = attn_partial_kernel<D, BITS, GQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.n_chunks, a.k.B * a.k.H, a.n_layers);
+  dim3 grid(a.n_chunks, a.k.B * a.k.H, a.n_layers);  // one CTA per split of kCpc chunks
   kern<<<grid, kAttnThreads, smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -485,7 +556,7 @@ uint64_t attn_workspace_bytes(const KvGeom& k, int hq, int n_layers, int n_token
 }
 
 cudaError_t launch_decode_attention(AttnArgs a, cudaStream_t st) {
-  a.n_chunks = (a.n_tokens + kChunk - 1) / kChunk;
+  a.n_chunks = ((a.n_tokens + kChunk - 1) / kChunk + kCpc - 1) / kCpc;  // partials per (layer, batch, query head)
   return a.k.d == 128 ? attn_bits<128>(a, st) : attn_bits<64>(a, st);
 }
 
