@@ -151,3 +151,77 @@ def test_zero_extremes_are_positive_zero():
     # a negative minimum keeps its sign, and a non-zero block is unchanged
     q, z, s = oq.quantize_ranges(np.array([[-0.5, 1.0]]), 4)
     assert z[0] == -0.5 and s[0] == fl16(fl32(1.5 / 15))
+
+
+def test_saturation_at_fp16_range():
+    """Ranges beyond fp16: the zero point clamps to -65504 (fp16's largest finite
+    magnitude), the step to 65504, and the codes then saturate.  Worked by hand at
+    4 bits (qmax 15): block [-1e6, 1e6] has fl32(2e6 / 15) = 133333.33 > 65504, so
+    z = -65504, s = 65504, inv = fl32(1 / 65504); -1e6 gives t < 0 -> 0, 1e6 gives
+    t = (1e6 + 65504) / 65504 = 16.27 -> 15, and 0 gives t = 1.0 -> 1."""
+    q, z, s = oq.quantize_ranges(np.array([[-1e6, 1e6, 0.0]]), 4)
+    assert z[0] == -65504.0 and s[0] == 65504.0
+    assert list(q[0]) == [0, 15, 1]
+    # a minimum below the range, a step inside it: z clamps, s does not
+    q, z, s = oq.quantize_ranges(np.array([[-70000.0, -69970.0]]), 4)
+    assert z[0] == -65504.0 and s[0] == fl16(fl32(30.0 / 15.0)) == 2.0
+    assert list(q[0]) == [0, 0]  # both below z: t < 0
+    # the largest step that is not clamped: (mx - mn) / 15 exactly 65504
+    q, z, s = oq.quantize_ranges(np.array([[0.0, 65504.0 * 15]]), 4)
+    assert z[0] == 0.0 and s[0] == 65504.0 and list(q[0]) == [0, 15]
+
+
+def test_metrics_hand_values():
+    """nrmse = ||x - xhat|| / ||x||, mse = mean squared error, max_abs, and bits/value
+    = 8 (code bytes + 4 bytes of fp16 step and zero per range) / values, on values
+    worked by hand."""
+    from oracle import metrics as om
+    x, xh = np.array([3.0, 4.0]), np.array([3.0, 0.0])
+    assert om.nrmse(x, xh) == 0.8          # sqrt(16) / sqrt(25)
+    assert om.mse(x, xh) == 8.0            # (0 + 16) / 2
+    assert om.max_abs(x, xh) == 4.0
+    assert om.nrmse(np.zeros(3), np.ones(3)) == 0.0  # zero reference: defined as 0
+    # 4 bits, 16 x 16 ranges: 128 code bytes and one range per 256 values -> 4.125
+    assert om.bits_per_value(128, 1, 256) == 4.125
+
+
+def test_kivi_views_by_index():
+    """kivi_key_view puts token 32 g + i of channel c at [g, c, i]; kivi_value_view puts
+    channel 32 g + i of token t at [t, g, i]; both unviews invert them exactly
+    (values that encode their own (t, c) index)."""
+    T, d = 64, 64
+    t = np.arange(T)[:, None]
+    c = np.arange(d)[None, :]
+    y = (1000 * t + c).astype(np.float64)[None]      # [1, T, d]
+    kv = oq.kivi_key_view(y, 32)                       # [1, T/32, d, 32]
+    assert kv.shape == (1, 2, 64, 32)
+    assert kv[0, 1, 5, 7] == 1000 * (32 + 7) + 5
+    assert kv[0, 0, 63, 31] == 1000 * 31 + 63
+    vv = oq.kivi_value_view(y, 32)                     # [1, T, d/32, 32]
+    assert vv.shape == (1, 64, 2, 32)
+    assert vv[0, 10, 1, 3] == 1000 * 10 + 32 + 3
+    assert np.array_equal(oq.kivi_key_unview(kv), y) and np.array_equal(oq.kivi_value_unview(vv), y)
+
+
+def test_kivi_exact_grid_encode_decode():
+    """An identity gauge on inputs whose ranges are exact grids: every key channel's 32
+    tokens take the values 0..7 (3 bits: z = 0, s = 1), every value token's 32 channels
+    too; the codes are then the values themselves, packed as the layout states, and the
+    decode returns the input exactly."""
+    L, B, H, T, d, bits = 1, 1, 1, 32, 32, 3
+    t = np.arange(T)[:, None]
+    c = np.arange(d)[None, :]
+    keys = ((t + c) % 8).astype(np.float64)            # each channel: 0..7 over its 32 tokens
+    vals = ((3 * c + t) % 8).astype(np.float64)        # each token: 0..7 over its 32 channels
+    x = np.stack([keys, vals])[None, :, None, None]    # [1, 2, 1, 1, T, d]
+    G = np.broadcast_to(np.eye(16), (L, 2, H, d // 16, 16, 16)).copy()
+    enc = oc.encode_kivi(x, G, bits)
+    assert np.all(enc["key"]["z"] == 0) and np.all(enc["key"]["s"] == 1)
+    assert np.all(enc["value"]["z"] == 0) and np.all(enc["value"]["s"] == 1)
+    assert np.array_equal(enc["key"]["q"][0, 0, 0, 0], keys.T)           # [channel][token]
+    assert np.array_equal(enc["value"]["q"][0, 0, 0, :, 0], vals)        # [token][channel]
+    # channel 0's key record: tokens 0..31 hold 0,1,..,7,0,.. -> 3-bit stream 0b..010001000
+    rec = enc["key"]["codes"][0, 0, 0, 0, 0]
+    assert rec.size == 12 and int.from_bytes(bytes(rec[:3]), "little") == sum(k << (3 * k) for k in range(8))
+    xr = oc.decode_kivi(enc, G, bits)
+    assert np.array_equal(xr, x)
