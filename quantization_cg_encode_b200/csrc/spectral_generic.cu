@@ -38,7 +38,7 @@ template <int D>
 struct GenSmem {
   static constexpr int P = D + 1;  // padded row pitch
   static constexpr int FLOATS = D * P /* C_d */ + 256 /* C_16 */ + 16 * D /* x */ + 2 * 16 * P /* two work */ +
-                                (D / 16) * 256 /* G */ + D /* radius columns */ + 3 * 8 + 8;
+                                (D / 16) * 256 /* G */ + D /* radius columns */ + 3 * 8 /* reductions */;
   static constexpr int BYTES = FLOATS * 4;
 };
 
@@ -75,7 +75,6 @@ __global__ void __launch_bounds__(kGenThreads) spectral_generic_kernel(GenArgs a
   float* Gs = w2 + 16 * P;        // [NG][16][16]
   float* rv = Gs + NG * 256;      // [D]: v / (d - 1)
   float* red = rv + D;            // [3][8]
-  float* blk = red + 24;          // [2]: L_freq and 1 / E of the block
   const int tid = threadIdx.x;
 
   for (int e = tid; e < D * D; e += kGenThreads) Cd[(e / D) * P + e % D] = dct_c(e / D, e % D, D);
