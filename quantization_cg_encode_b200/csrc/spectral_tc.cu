@@ -32,6 +32,8 @@
 // [256,384) dU1^T, [384,512) dM.  Every mbarrier wait is bounded in time.
 #include <cuda.h>
 
+#include <utility>
+
 #include "cg_kernels.cuh"
 
 namespace cg {
@@ -75,6 +77,104 @@ constexpr C16Table make_c16() {
   return c;
 }
 __constant__ C16Table c16t = make_c16();
+
+// Compile-time loop: the body sees its index as a constant expression, so the
+// DCT coefficients below become immediates.
+template <typename F, int... I>
+__device__ __forceinline__ void unroll_seq(F&& f, std::integer_sequence<int, I...>) {
+  (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void unroll_n(F&& f) {
+  unroll_seq(f, std::make_integer_sequence<int, N>{});
+}
+__device__ __forceinline__ float2 dup2(float c) { return make_float2(c, c); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, dup2(-1.0f), a); }
+// log2 of an argument >= 1 (never subnormal, so flushing changes nothing)
+__device__ __forceinline__ float lg2_ftz(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 16-point orthonormal DCT-II of two token blocks at once (block A in .x, block B
+// in .y), by partial butterflies on the symmetry C_16[u][15 - t] = (-1)^u C_16[u][t]:
+// sums a and differences b of mirrored tokens; the odd frequencies are the 8 x 8
+// half of C_16 on b; the even ones an 8-point DCT of a, split the same way twice
+// (c, e = a[t] +- a[7 - t]; f, g = c[t] +- c[3 - t]).  100 paired operations per
+// 32 coefficients against 256 scalar ones for the plain matrix product.
+__device__ __forceinline__ void dct16_pair(const float* sa, const float* sb, float2 (&U)[16]) {
+  float2 a[8], b[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    a[t] = make_float2(sa[t] + sa[15 - t], sb[t] + sb[15 - t]);
+    b[t] = make_float2(sa[t] - sa[15 - t], sb[t] - sb[15 - t]);
+  }
+  unroll_n<8>([&](auto k) {  // u = 1, 3, .., 15
+    constexpr int u = 2 * decltype(k)::value + 1;
+    constexpr float c0 = c16_value(u, 0);
+    float2 acc = __fmul2_rn(dup2(c0), b[0]);
+    unroll_n<7>([&](auto t1) {
+      constexpr int t = decltype(t1)::value + 1;
+      constexpr float ct = c16_value(u, t);
+      acc = __ffma2_rn(dup2(ct), b[t], acc);
+    });
+    U[u] = acc;
+  });
+  float2 c[4], e[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    c[t] = __fadd2_rn(a[t], a[7 - t]);
+    e[t] = sub2(a[t], a[7 - t]);
+  }
+  unroll_n<4>([&](auto k) {  // u = 2, 6, 10, 14
+    constexpr int u = 4 * decltype(k)::value + 2;
+    constexpr float c0 = c16_value(u, 0);
+    float2 acc = __fmul2_rn(dup2(c0), e[0]);
+    unroll_n<3>([&](auto t1) {
+      constexpr int t = decltype(t1)::value + 1;
+      constexpr float ct = c16_value(u, t);
+      acc = __ffma2_rn(dup2(ct), e[t], acc);
+    });
+    U[u] = acc;
+  });
+  const float2 f0 = __fadd2_rn(c[0], c[3]), f1 = __fadd2_rn(c[1], c[2]);
+  const float2 g0 = sub2(c[0], c[3]), g1 = sub2(c[1], c[2]);
+  unroll_n<2>([&](auto k) {  // u = 4, 12
+    constexpr int u = 8 * decltype(k)::value + 4;
+    constexpr float c0 = c16_value(u, 0), c1 = c16_value(u, 1);
+    U[u] = __ffma2_rn(dup2(c1), g1, __fmul2_rn(dup2(c0), g0));
+  });
+  U[0] = __fmul2_rn(dup2(0.25f), __fadd2_rn(f0, f1));  // C_16[0][t] = 1/4
+  U[8] = __fmul2_rn(dup2(0.25f), sub2(f0, f1));        // C_16[8][t] = 1/4, -1/4 for t = 0, 1
+}
+
+// Per-block sums over the 16 frequencies of a thread's channel frequency v, for the
+// two blocks of a pair: E = sum U^2, F = sum r_uv U^2, R = sum log2(1 + |U| / tau)
+// (the logarithms taken two at a time, log2 p + log2 q = log2 (p q)).
+__device__ __forceinline__ void pair_sums(const float2 (&U)[16], const float2 (&rad2)[16], float inv_tau, float2& E,
+                                          float2& F, float2& R) {
+  float2 pr = make_float2(1.0f, 1.0f);
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const float2 e2 = __fmul2_rn(U[u], U[u]);
+    if (u == 0) {
+      E = e2;
+      F = __fmul2_rn(rad2[0], e2);
+    } else {
+      E = __fadd2_rn(E, e2);
+      F = __ffma2_rn(rad2[u], e2, F);
+    }
+    const float2 g = make_float2(__fmaf_rn(fabsf(U[u].x), inv_tau, 1.0f), __fmaf_rn(fabsf(U[u].y), inv_tau, 1.0f));
+    if (u & 1) {
+      const float2 q = __fmul2_rn(pr, g);
+      const float2 l = make_float2(lg2_ftz(q.x), lg2_ftz(q.y));
+      R = u == 1 ? l : __fadd2_rn(R, l);
+    } else {
+      pr = g;
+    }
+  }
+}
 
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) {  // K-major, 128-byte swizzle
   uint64_t d = (uint64_t)((addr & 0x3FFFFu) >> 4);
@@ -347,13 +447,13 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
     const int v = 32 * wq + lane;
     const uint32_t lrow = (uint32_t)(32 * wq) << 16;
     const float inv_tau = 1.0f / a.tau;
-    float rad[16];
+    float2 rad2[16];
     {
       const float rv = (float)v / (kD - 1);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const float ru = (float)u / 15.0f;
-        rad[u] = sqrtf(ru * ru + rv * rv) * 0.70710678118654752f;
+        rad2[u] = dup2(sqrtf(ru * ru + rv * rv) * 0.70710678118654752f);
       }
     }
     int i = 0;
@@ -396,32 +496,23 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
         __syncwarp();
         if (lane == 0) mbar_arrive(u_empty);
         // token DCT of the four 16-token blocks (even / odd halves), and this v's share of the sums
-        float part[12];  // per block: sum U^2, sum r U^2, sum log2(1 + |U|/tau)
+        float part[12];  // per block kb: sum U^2, sum r U^2, sum log2(1 + |U|/tau) at 3 kb
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          float* col = x + 16 * kb;
-          float sm8[8], df8[8];
+        for (int p = 0; p < 2; ++p) {  // blocks 2 p and 2 p + 1 as fp32 pairs
+          float2 U[16], E, F, R;
+          dct16_pair(x + 32 * p, x + 32 * p + 16, U);
+          pair_sums(U, rad2, inv_tau, E, F, R);
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            sm8[t] = col[t] + col[15 - t];
-            df8[t] = col[t] - col[15 - t];
+          for (int u = 0; u < 16; ++u) {  // U in place of the blocks' columns
+            x[32 * p + u] = U[u].x;
+            x[32 * p + 16 + u] = U[u].y;
           }
-          float e = 0.0f, f = 0.0f, rr = 0.0f, pr = 1.0f;
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            float acc = c16t.v[u][0] * ((u & 1) ? df8[0] : sm8[0]);
-#pragma unroll
-            for (int t = 1; t < 8; ++t) acc = __fmaf_rn(c16t.v[u][t], (u & 1) ? df8[t] : sm8[t], acc);
-            col[u] = acc;  // U[u], in place of the block's column (its inputs live in sm8 / df8)
-            const float e2 = acc * acc;
-            e += e2;
-            f = __fmaf_rn(rad[u], e2, f);
-            if (u & 1) rr += __log2f(pr * __fmaf_rn(fabsf(acc), inv_tau, 1.0f));
-            else pr = __fmaf_rn(fabsf(acc), inv_tau, 1.0f);
-          }
-          part[3 * kb] = e;
-          part[3 * kb + 1] = f;
-          part[3 * kb + 2] = rr;
+          part[6 * p] = E.x;
+          part[6 * p + 1] = F.x;
+          part[6 * p + 2] = R.x;
+          part[6 * p + 3] = E.y;
+          part[6 * p + 4] = F.y;
+          part[6 * p + 5] = R.y;
         }
 #pragma unroll
         for (int q = 0; q < 12; ++q) {
@@ -465,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
           for (int u = 0; u < 16; ++u) {
             const float U = x[16 * kb + u];
             const float sg = U > 0.0f ? 1.0f : (U < 0.0f ? -1.0f : 0.0f);
-            dU[u] = __fmaf_rn(cf * U, rad[u] - lf[kb], __fdividef(cr * sg, a.tau + fabsf(U)));
+            dU[u] = __fmaf_rn(cf * U, rad2[u].x - lf[kb], __fdividef(cr * sg, a.tau + fabsf(U)));
           }
           float d1[16];
 #pragma unroll
@@ -693,13 +784,13 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
     const int v = 32 * wq + lane;
     const uint32_t lrow = (uint32_t)(32 * wq) << 16;
     const float inv_tau = 1.0f / a.tau;
-    float rad[16];
+    float2 rad2[16];
     {
       const float rv = (float)v / (kD - 1);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const float ru = (float)u / 15.0f;
-        rad[u] = sqrtf(ru * ru + rv * rv) * 0.70710678118654752f;
+        rad2[u] = dup2(sqrtf(ru * ru + rv * rv) * 0.70710678118654752f);
       }
     }
     int ls = -1;
@@ -739,31 +830,18 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&u_empty[ub]);
-      float part[12];
+      float part[12];  // per block kb: E, F, R at 3 kb
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        const float* col = x + 16 * kb;
-        float sm8[8], df8[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          sm8[t] = col[t] + col[15 - t];
-          df8[t] = col[t] - col[15 - t];
-        }
-        float e = 0.0f, f = 0.0f, rr = 0.0f, pr = 1.0f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          float U = c16t.v[u][0] * ((u & 1) ? df8[0] : sm8[0]);
-#pragma unroll
-          for (int t = 1; t < 8; ++t) U = __fmaf_rn(c16t.v[u][t], (u & 1) ? df8[t] : sm8[t], U);
-          const float e2 = U * U;
-          e += e2;
-          f = __fmaf_rn(rad[u], e2, f);
-          if (u & 1) rr += __log2f(pr * __fmaf_rn(fabsf(U), inv_tau, 1.0f));
-          else pr = __fmaf_rn(fabsf(U), inv_tau, 1.0f);
-        }
-        part[3 * kb] = e;
-        part[3 * kb + 1] = f;
-        part[3 * kb + 2] = rr;
+      for (int p = 0; p < 2; ++p) {  // blocks 2 p and 2 p + 1 as fp32 pairs
+        float2 U[16], E, F, R;
+        dct16_pair(x + 32 * p, x + 32 * p + 16, U);
+        pair_sums(U, rad2, inv_tau, E, F, R);
+        part[6 * p] = E.x;
+        part[6 * p + 1] = F.x;
+        part[6 * p + 2] = R.x;
+        part[6 * p + 3] = E.y;
+        part[6 * p + 4] = F.y;
+        part[6 * p + 5] = R.y;
       }
       const float tot = warp_sum12(part, lane);
       float* rb = red + ((i & 1) * 2 + hf) * 48;
