@@ -629,11 +629,14 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
 // into contiguous ranges, one per CTA (a range may start inside a slice and
 // cross into the next ones, each with its own gauge), instead of whole slices,
 // and U1^T is double-buffered in tensor memory so the GEMM of tile i + 1 runs
-// while the workers take tile i's token DCT and statistics.  Tensor memory:
-// [0,128) M (bf16 hi, lo), [128,256) and [256,384) U1^T.
+// while the workers take tile i's token DCT and statistics.  M is double-buffered
+// too: the workers build the next slice's M before the current slice's last tile,
+// so the GEMM of the next slice's first tile overlaps that tile's statistics.
+// Tensor memory: [0,128) and [384,512) M (bf16 hi, lo), [128,256) and [256,384) U1^T.
 namespace {
 
-constexpr uint32_t kFColM = 0, kFColU1 = 128;
+constexpr uint32_t kFColM0 = 0, kFColM1 = 384, kFColU1 = 128;
+__device__ __forceinline__ uint32_t fwd_mcol(int q) { return (q & 1) ? kFColM1 : kFColM0; }
 constexpr int kFwdSmem = 1024 + kStages * kXBytes + 2 * 8192 + 2 * 2 * 4 * 12 * 4 + kCosTab * 4 + 256;
 
 // Sum of 12 per-lane values over a warp: afterwards lane l holds the total of
@@ -675,9 +678,9 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
   uint64_t* x_empty = bars + kStages;
   uint64_t* g_full = bars + 2 * kStages;  // [2]
   uint64_t* g_empty = g_full + 2;         // [2]
-  uint64_t* m_full = g_empty + 2;
-  uint64_t* m_empty = m_full + 1;
-  uint64_t* u_full = m_empty + 1;         // [2]
+  uint64_t* m_full = g_empty + 2;         // [2]
+  uint64_t* m_empty = m_full + 2;         // [2]
+  uint64_t* u_full = m_empty + 2;         // [2]
   uint64_t* u_empty = u_full + 2;         // [2]
   uint64_t* mma_done = u_empty + 2;
   uint32_t* tmem_base = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -704,8 +707,10 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
       mbar_init(&u_full[s], 1);
       mbar_init(&u_empty[s], kWorkerWarps);
     }
-    mbar_init(m_full, kWorkerWarps);
-    mbar_init(m_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&m_full[s], kWorkerWarps);
+      mbar_init(&m_empty[s], 1);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
     fence_mbar_init();
@@ -759,22 +764,24 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
         const int j = (int)(gt % tiles), s = i % kStages, ub = i & 1;
         if (i == 0 || j == 0) {
           ++lsm;
-          if (a.has_g || i == 0) wait(m_full, (uint32_t)(a.has_g ? lsm : 0) & 1u);
+          // slice lsm's M (with a gauge, buffer lsm & 1; without, one M in buffer 0)
+          if (a.has_g || i == 0) wait(&m_full[lsm & 1], (uint32_t)(a.has_g ? lsm >> 1 : 0) & 1u);
         }
         wait(&x_full[s], (uint32_t)(i / kStages) & 1u);
         wait(&u_empty[ub], ((uint32_t)(i >> 1) & 1u) ^ 1u);
         fence_after();
         const uint32_t xa = smem_u32(xs + s * kXBytes);
         const uint32_t d = tmem + kFColU1 + 128 * ub;
+        const uint32_t mc = tmem + fwd_mcol(a.has_g ? lsm : 0);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint64_t bd = kdesc(xa + (k >> 2) * 16384 + (k & 3) * 32);
-          mma_ts(d, tmem + kFColM + 8 * k, bd, idesc(false), k > 0);
-          mma_ts(d, tmem + kFColM + 64 + 8 * k, bd, idesc(false), 1);
+          mma_ts(d, mc + 8 * k, bd, idesc(false), k > 0);
+          mma_ts(d, mc + 64 + 8 * k, bd, idesc(false), 1);
         }
         commit(&u_full[ub]);
         commit(&x_empty[s]);
-        if (a.has_g && (j == tiles - 1 || i == n_t - 1)) commit(m_empty);
+        if (a.has_g && (j == tiles - 1 || i == n_t - 1)) commit(&m_empty[lsm & 1]);
       }
       commit(mma_done);
       mbar_wait(mma_done, 0u, a.status);
@@ -793,33 +800,39 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
         rad2[u] = dup2(sqrtf(ru * ru + rv * rv) * 0.70710678118654752f);
       }
     }
-    int ls = -1;
+    // M of the q-th slice of this CTA's range into buffer q & 1, once that buffer's
+    // previous slice (q - 2) has had all its GEMMs
+    auto build_m = [&](int q) {
+      if (a.has_g) wait(&g_full[q & 1], (uint32_t)(q >> 1) & 1u);
+      if (q >= 2) wait(&m_empty[q & 1], (uint32_t)((q - 2) >> 1) & 1u);
+      __syncwarp();
+      fence_after();
+      const float* G = gs + (q & 1) * 2048;
+      const uint32_t mc = tmem + lrow + fwd_mcol(q);
+#pragma unroll 1
+      for (int r4 = 0; r4 < 4; ++r4) {
+        const int r = 4 * hf + r4;
+        uint32_t h8[8], l8[8];
+        m_group(cosk, G, a.has_g, v, r, h8, l8);
+        st8(mc + 8 * r, h8);
+        st8(mc + 64 + 8 * r, l8);
+      }
+      wait_st();
+      fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&m_full[q & 1]);
+        if (a.has_g) mbar_arrive(&g_empty[q & 1]);
+      }
+    };
+    if (n_t > 0) build_m(0);
+    int ls = 0;
     for (int i = 0; i < n_t; ++i) {
       const long long gt = g0 + i;
       const int j = (int)(gt % tiles), ub = i & 1;
-      if (i == 0 || j == 0) ++ls;
-      if ((i == 0 || j == 0) && (a.has_g || i == 0)) {
-        if (a.has_g) wait(&g_full[ls & 1], (uint32_t)(ls >> 1) & 1u);
-        if (a.has_g && ls > 0) wait(m_empty, (uint32_t)(ls - 1) & 1u);
-        __syncwarp();
-        fence_after();
-        const float* G = gs + (ls & 1) * 2048;
-#pragma unroll 1
-        for (int r4 = 0; r4 < 4; ++r4) {
-          const int r = 4 * hf + r4;
-          uint32_t h8[8], l8[8];
-          m_group(cosk, G, a.has_g, v, r, h8, l8);
-          st8(tmem + lrow + kFColM + 8 * r, h8);
-          st8(tmem + lrow + kFColM + 64 + 8 * r, l8);
-        }
-        wait_st();
-        fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(m_full);
-          if (a.has_g) mbar_arrive(&g_empty[ls & 1]);
-        }
-      }
+      if (i > 0 && j == 0) ++ls;
+      // the next tile starts a slice: its M now, before this tile's statistics
+      if (a.has_g && i + 1 < n_t && j == tiles - 1) build_m(ls + 1);
       wait(&u_full[ub], (uint32_t)(i >> 1) & 1u);
       __syncwarp();
       fence_after();
