@@ -67,16 +67,6 @@ constexpr float c16_value(int u, int t) {
   }
   return u == 0 ? 0.25f : sg * kCosPi32[k];
 }
-struct C16Table {
-  float v[16][8];
-};
-constexpr C16Table make_c16() {
-  C16Table c{};
-  for (int u = 0; u < 16; ++u)
-    for (int t = 0; t < 8; ++t) c.v[u][t] = c16_value(u, t);
-  return c;
-}
-__constant__ C16Table c16t = make_c16();
 
 // Compile-time loop: the body sees its index as a constant expression, so the
 // DCT coefficients below become immediates.
@@ -149,6 +139,54 @@ __device__ __forceinline__ void dct16_pair(const float* sa, const float* sb, flo
   U[8] = __fmul2_rn(dup2(0.25f), sub2(f0, f1));        // C_16[8][t] = 1/4, -1/4 for t = 0, 1
 }
 
+// The transpose of dct16_pair, s[t] = sum_u C_16[u][t] dU[u] for two blocks at once: the
+// same butterflies taken backwards (odd frequencies onto the differences b, u = 2 mod 4
+// onto e, u = 4, 12 onto g, u = 0, 8 onto f, then the sums and differences undone).
+__device__ __forceinline__ void idct16_pair(const float2 (&dU)[16], float2 (&s)[16]) {
+  float2 db[8], de[4], dg[2];
+  unroll_n<8>([&](auto tt) {
+    constexpr int t = decltype(tt)::value;
+    constexpr float c1 = c16_value(1, t);
+    float2 acc = __fmul2_rn(dup2(c1), dU[1]);
+    unroll_n<7>([&](auto k1) {
+      constexpr int u = 2 * decltype(k1)::value + 3;
+      constexpr float cu = c16_value(u, t);
+      acc = __ffma2_rn(dup2(cu), dU[u], acc);
+    });
+    db[t] = acc;
+  });
+  unroll_n<4>([&](auto tt) {
+    constexpr int t = decltype(tt)::value;
+    constexpr float c2 = c16_value(2, t);
+    float2 acc = __fmul2_rn(dup2(c2), dU[2]);
+    unroll_n<3>([&](auto k1) {
+      constexpr int u = 4 * decltype(k1)::value + 6;
+      constexpr float cu = c16_value(u, t);
+      acc = __ffma2_rn(dup2(cu), dU[u], acc);
+    });
+    de[t] = acc;
+  });
+  unroll_n<2>([&](auto tt) {
+    constexpr int t = decltype(tt)::value;
+    constexpr float c4 = c16_value(4, t), c12 = c16_value(12, t);
+    dg[t] = __ffma2_rn(dup2(c12), dU[12], __fmul2_rn(dup2(c4), dU[4]));
+  });
+  const float2 df0 = __fmul2_rn(dup2(0.25f), __fadd2_rn(dU[0], dU[8]));
+  const float2 df1 = __fmul2_rn(dup2(0.25f), sub2(dU[0], dU[8]));
+  const float2 dc[4] = {__fadd2_rn(df0, dg[0]), __fadd2_rn(df1, dg[1]), sub2(df1, dg[1]), sub2(df0, dg[0])};
+  float2 da[8];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    da[t] = __fadd2_rn(dc[t], de[t]);
+    da[7 - t] = sub2(dc[t], de[t]);
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    s[t] = __fadd2_rn(da[t], db[t]);
+    s[15 - t] = sub2(da[t], db[t]);
+  }
+}
+
 // Per-block sums over the 16 frequencies of a thread's channel frequency v, for the
 // two blocks of a pair: E = sum U^2, F = sum r_uv U^2, R = sum log2(1 + |U| / tau)
 // (the logarithms taken two at a time, log2 p + log2 q = log2 (p q)).
@@ -174,6 +212,31 @@ __device__ __forceinline__ void pair_sums(const float2 (&U)[16], const float2 (&
       pr = g;
     }
   }
+}
+
+// Sum of 12 per-lane values over a warp: afterwards lane l holds the total of
+// value l >> 1 (l >> 1 < 12).  Each exchange halves the values a lane carries.
+__device__ __forceinline__ float warp_sum12(const float (&p)[12], int lane) {
+  float a8[8], a4[4], a2[2];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const float lo = p[m], hi = m + 8 < 12 ? p[m + 8] : 0.0f;
+    const bool up = lane & 16;
+    a8[m] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, 16);
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const bool up = lane & 8;
+    a4[m] = (up ? a8[m + 4] : a8[m]) + __shfl_xor_sync(0xffffffffu, up ? a8[m] : a8[m + 4], 8);
+  }
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const bool up = lane & 4;
+    a2[m] = (up ? a4[m + 2] : a4[m]) + __shfl_xor_sync(0xffffffffu, up ? a4[m] : a4[m + 2], 4);
+  }
+  const bool up = lane & 2;
+  float r = (up ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, up ? a2[0] : a2[1], 2);
+  return r + __shfl_xor_sync(0xffffffffu, r, 1);
 }
 
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) {  // K-major, 128-byte swizzle
@@ -514,16 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
           part[6 * p + 4] = F.y;
           part[6 * p + 5] = R.y;
         }
-#pragma unroll
-        for (int q = 0; q < 12; ++q) {
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) part[q] += __shfl_xor_sync(0xffffffffu, part[q], o);
-        }
+        const float tot = warp_sum12(part, lane);
         float* rb = red + ((i & 1) * 2 + hf) * 48;  // [quarter][12] of this tile parity and half
-        if (lane == 0) {
-#pragma unroll
-          for (int q = 0; q < 12; ++q) rb[wq * 12 + q] = part[q];
-        }
+        if (!(lane & 1) && (lane >> 1) < 12) rb[wq * 12 + (lane >> 1)] = tot;
         named_bar_sync(2 + hf, 128);
         float E[4], F[4], R[4], lf[4];
 #pragma unroll
@@ -549,32 +605,33 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
         const float cr = (float)(a.lambda_r * a.inv_ncoef);
         const float cf0 = (float)(2.0 * a.lambda_f * a.inv_nblk);
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          const float cf = E[kb] > 0.0f ? __fdividef(cf0, E[kb]) : 0.0f;
-          float dU[16];
+        for (int p = 0; p < 2; ++p) {  // blocks 2 p and 2 p + 1 as fp32 pairs
+          float2 dU[16], d1[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float U = x[16 * kb + u];
-            const float sg = U > 0.0f ? 1.0f : (U < 0.0f ? -1.0f : 0.0f);
-            dU[u] = __fmaf_rn(cf * U, rad2[u].x - lf[kb], __fdividef(cr * sg, a.tau + fabsf(U)));
-          }
-          float d1[16];
+          for (int h = 0; h < 2; ++h) {
+            const int kb = 2 * p + h;
+            const float cf = E[kb] > 0.0f ? __fdividef(cf0, E[kb]) : 0.0f;
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            float ev = 0.0f, od = 0.0f;
-#pragma unroll
-            for (int u = 0; u < 16; u += 2) {
-              ev = __fmaf_rn(c16t.v[u][t], dU[u], ev);
-              od = __fmaf_rn(c16t.v[u + 1][t], dU[u + 1], od);
+            for (int u = 0; u < 16; ++u) {
+              const float U = x[16 * kb + u];
+              const float sg = U > 0.0f ? 1.0f : (U < 0.0f ? -1.0f : 0.0f);
+              const float g = __fmaf_rn(cf * U, rad2[u].x - lf[kb], __fdividef(cr * sg, a.tau + fabsf(U)));
+              if (h == 0) dU[u].x = g;
+              else dU[u].y = g;
             }
-            d1[t] = ev + od;
-            d1[15 - t] = ev - od;
           }
-          uint32_t h8[8], l8[8];
+          idct16_pair(dU, d1);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) split2(d1[2 * q], d1[2 * q + 1], h8[q], l8[q]);
-          st8(tmem + lrow + kColDU + 32 * hf + 8 * kb, h8);
-          st8(tmem + lrow + kColDU + 64 + 32 * hf + 8 * kb, l8);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t h8[8], l8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float2 e0 = d1[2 * q], e1 = d1[2 * q + 1];
+              split2(h ? e0.y : e0.x, h ? e1.y : e1.x, h8[q], l8[q]);
+            }
+            st8(tmem + lrow + kColDU + 32 * hf + 8 * (2 * p + h), h8);
+            st8(tmem + lrow + kColDU + 64 + 32 * hf + 8 * (2 * p + h), l8);
+          }
         }
         wait_st();
         fence_before();
@@ -637,32 +694,9 @@ namespace {
 
 constexpr uint32_t kFColM0 = 0, kFColM1 = 384, kFColU1 = 128;
 __device__ __forceinline__ uint32_t fwd_mcol(int q) { return (q & 1) ? kFColM1 : kFColM0; }
-constexpr int kFwdSmem = 1024 + kStages * kXBytes + 2 * 8192 + 2 * 2 * 4 * 12 * 4 + kCosTab * 4 + 256;
+constexpr int kRedPitch = 132;  // [12][kRedPitch] partial sums of a tile half, by channel frequency v
+constexpr int kFwdSmem = 1024 + kStages * kXBytes + 2 * 8192 + 2 * 2 * 12 * kRedPitch * 4 + kCosTab * 4 + 256;
 
-// Sum of 12 per-lane values over a warp: afterwards lane l holds the total of
-// value l >> 1 (l >> 1 < 12).  Each exchange halves the values a lane carries.
-__device__ __forceinline__ float warp_sum12(const float (&p)[12], int lane) {
-  float a8[8], a4[4], a2[2];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const float lo = p[m], hi = m + 8 < 12 ? p[m + 8] : 0.0f;
-    const bool up = lane & 16;
-    a8[m] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, 16);
-  }
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const bool up = lane & 8;
-    a4[m] = (up ? a8[m + 4] : a8[m]) + __shfl_xor_sync(0xffffffffu, up ? a8[m] : a8[m + 4], 8);
-  }
-#pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const bool up = lane & 4;
-    a2[m] = (up ? a4[m + 2] : a4[m]) + __shfl_xor_sync(0xffffffffu, up ? a4[m] : a4[m + 2], 4);
-  }
-  const bool up = lane & 2;
-  float r = (up ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, up ? a2[0] : a2[1], 2);
-  return r + __shfl_xor_sync(0xffffffffu, r, 1);
-}
 
 }  // namespace
 
@@ -671,8 +705,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
   unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char* xs = base;                                      // ring of x tiles
   float* gs = reinterpret_cast<float*>(xs + kStages * kXBytes);  // 2 x [8][16][16] G
-  float* red = reinterpret_cast<float*>(gs + 2 * 2048);          // [2 tile parity][2 half][4 quarter][12]
-  float* cosk = red + 2 * 2 * 4 * 12;                            // cos(k pi / 256)
+  float* red = reinterpret_cast<float*>(gs + 2 * 2048);          // [2 tile parity][2 half][12][kRedPitch]
+  float* cosk = red + 2 * 2 * 12 * kRedPitch;                    // cos(k pi / 256)
   uint64_t* bars = reinterpret_cast<uint64_t*>(cosk + kCosTab);
   uint64_t* x_full = bars;
   uint64_t* x_empty = bars + kStages;
@@ -856,18 +890,29 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
         part[6 * p + 4] = F.y;
         part[6 * p + 5] = R.y;
       }
-      const float tot = warp_sum12(part, lane);
-      float* rb = red + ((i & 1) * 2 + hf) * 48;
-      if (!(lane & 1) && (lane >> 1) < 12) rb[wq * 12 + (lane >> 1)] = tot;
+      float* rb = red + ((i & 1) * 2 + hf) * (12 * kRedPitch);
+#pragma unroll
+      for (int q = 0; q < 12; ++q) rb[q * kRedPitch + v] = part[q];
       named_bar_sync(2 + hf, 128);
-      if (wq == 0 && lane < 4) {
-        const int kb = lane;
-        const float E = (rb[0 * 12 + 3 * kb] + rb[1 * 12 + 3 * kb]) + (rb[2 * 12 + 3 * kb] + rb[3 * 12 + 3 * kb]);
-        const float F = (rb[0 * 12 + 3 * kb + 1] + rb[1 * 12 + 3 * kb + 1]) + (rb[2 * 12 + 3 * kb + 1] + rb[3 * 12 + 3 * kb + 1]);
-        const float R = (rb[0 * 12 + 3 * kb + 2] + rb[1 * 12 + 3 * kb + 2]) + (rb[2 * 12 + 3 * kb + 2] + rb[3 * 12 + 3 * kb + 2]);
-        const long long blk = gt * 8 + 4 * hf + kb;
-        a.lfreq[blk] = E > 0.0f ? F / E : 0.0f;
-        a.lrate[blk] = R * 0.69314718055994531f / (16.0f * kD);
+      // One warp per half (channel quarter 3 or 2: not the SMSPs of the producer and MMA
+      // warps) finishes the sums: lane 8 kb + s adds v = 16 s .. 16 s + 15 of block kb.
+      if (wq == (hf ? 2 : 3)) {
+        const int kb = lane >> 3, sx = lane & 7;
+        float acc[3];
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          const float4* src = reinterpret_cast<const float4*>(rb + (3 * kb + c) * kRedPitch + 16 * sx);
+          const float4 a0 = src[0], a1 = src[1], a2 = src[2], a3 = src[3];
+          acc[c] = (((a0.x + a0.y) + (a0.z + a0.w)) + ((a1.x + a1.y) + (a1.z + a1.w))) +
+                   (((a2.x + a2.y) + (a2.z + a2.w)) + ((a3.x + a3.y) + (a3.z + a3.w)));
+#pragma unroll
+          for (int o = 1; o < 8; o <<= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
+        }
+        if (sx == 0) {
+          const long long blk = gt * 8 + 4 * hf + kb;
+          a.lfreq[blk] = acc[0] > 0.0f ? acc[1] / acc[0] : 0.0f;
+          a.lrate[blk] = acc[2] * 0.69314718055994531f / (16.0f * kD);
+        }
       }
     }
   }
