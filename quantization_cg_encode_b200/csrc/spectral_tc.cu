@@ -47,7 +47,7 @@ constexpr int kThreads = (2 + kWorkerWarps) * 32;
 constexpr uint32_t kColU = 0, kColM = 128, kColDU = 256, kColDM = 384;
 constexpr int kDmPitch = kD + 1;
 // smem: 1024 align + ring + 2 G + dM staging + reductions + barriers
-constexpr int kSmem = 1024 + kStages * kXBytes + 2 * 8192 + kD * kDmPitch * 4 + 2 * 2 * 4 * 12 * 4 + 132 * 4 + 256;
+constexpr int kSmem = 1024 + kStages * kXBytes + 2 * 8192 + kD * kDmPitch * 4 + 2 * 2 * 4 * 12 * 4 + 2 * 512 * 4 + 256;
 
 // Orthonormal DCT-II coefficients C_16[u][t] for t < 8 (the other half follows
 // from C_16[u][15 - t] = (-1)^u C_16[u][t]): 1/4 for u = 0, else
@@ -296,44 +296,55 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
 }
 // Orthonormal DCT-II C_d[v][c] (d = 128) from cosk[k] = cos(k pi / 256), k = 0..128,
 // a table each CTA fills once: the angle (2 c + 1) v pi / 256 is folded onto [0, pi / 2].
-constexpr int kCosTab = 132;  // 129 entries, padded
+constexpr int kCosTab = 2 * 512;  // cos(k pi / 256) for a full period, each entry twice (a packed pair)
 __device__ __forceinline__ float cd_tab(const float* cosk, int v, int c) {
-  int k = ((2 * c + 1) * v) & 511;  // period 2 pi = 512 steps
-  if (k > 256) k = 512 - k;         // cos(2 pi - a) = cos a
-  const float cv = k > 128 ? -cosk[256 - k] : cosk[k];  // cos(pi - a) = -cos a
-  return (v == 0 ? 0.08838834764831845f : 0.125f) * cv;  // sqrt(1/128), sqrt(2/128)
+  return (v == 0 ? 0.08838834764831845f : 0.125f) * cosk[2 * (((2 * c + 1) * v) & 511)];  // sqrt(1/128), sqrt(2/128)
 }
-__device__ __forceinline__ void fill_cos_table(float* cosk, int wid) {
-  if (wid <= 128) cosk[wid] = cospif((float)wid / 256.0f);
+__device__ __forceinline__ void fill_cos_table(float* cosk, int wid) {  // wid = 0 .. 255
+  for (int k = wid; k < 512; k += 256) {
+    const float c = cospif((float)k / 256.0f);
+    cosk[2 * k] = c;
+    cosk[2 * k + 1] = c;
+  }
 }
 // Channels 16 r .. 16 r + 15 of row v of M = C_d blockdiag(G) (C_d alone without a
 // gauge), M[v][16 r + j] = sum_i C_d[v][16 r + i] G_r[i][j], as bf16 hi / lo pairs.
+// The angle index (2 c + 1) v steps by 2 v from one channel to the next; the products
+// run on fp32 pairs (two output channels per instruction).
 __device__ __forceinline__ void m_group(const float* cosk, const float* G, bool has_g, int v, int r, uint32_t (&h8)[8],
                                         uint32_t (&l8)[8]) {
-  float cd[16], m16[16];
-#pragma unroll
-  for (int ii = 0; ii < 16; ++ii) cd[ii] = cd_tab(cosk, v, 16 * r + ii);
+  const float2 sc = dup2(v == 0 ? 0.08838834764831845f : 0.125f);
+  const float2* cos2 = reinterpret_cast<const float2*>(cosk);
+  int k = ((32 * r + 1) * v) & 511;
+  float2 m2[8];
   if (has_g) {
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) m16[jj] = 0.0f;
-#pragma unroll
     for (int ii = 0; ii < 16; ++ii) {
+      const float2 cc = cos2[k];
+      k = (k + 2 * v) & 511;
       const float4* row = reinterpret_cast<const float4*>(G + (r * 16 + ii) * 16);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float4 g = row[q];
-        m16[4 * q] = __fmaf_rn(cd[ii], g.x, m16[4 * q]);
-        m16[4 * q + 1] = __fmaf_rn(cd[ii], g.y, m16[4 * q + 1]);
-        m16[4 * q + 2] = __fmaf_rn(cd[ii], g.z, m16[4 * q + 2]);
-        m16[4 * q + 3] = __fmaf_rn(cd[ii], g.w, m16[4 * q + 3]);
+        const float2 g01 = make_float2(g.x, g.y), g23 = make_float2(g.z, g.w);
+        m2[2 * q] = ii == 0 ? __fmul2_rn(cc, g01) : __ffma2_rn(cc, g01, m2[2 * q]);
+        m2[2 * q + 1] = ii == 0 ? __fmul2_rn(cc, g23) : __ffma2_rn(cc, g23, m2[2 * q + 1]);
       }
     }
   } else {
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) m16[jj] = cd[jj];
+    for (int q = 0; q < 8; ++q) {
+      const float c0 = cos2[k].x;
+      k = (k + 2 * v) & 511;
+      m2[q] = make_float2(c0, cos2[k].x);
+      k = (k + 2 * v) & 511;
+    }
   }
 #pragma unroll
-  for (int q = 0; q < 8; ++q) split2(m16[2 * q], m16[2 * q + 1], h8[q], l8[q]);
+  for (int q = 0; q < 8; ++q) {
+    const float2 m = __fmul2_rn(sc, m2[q]);
+    split2(m.x, m.y, h8[q], l8[q]);
+  }
 }
 
 struct TmArgs {
