@@ -130,9 +130,11 @@ def test_gauge_build_group_and_full_head():
     """cg_gauge_build against the oracle's fp64 exp(A - A^T), fp64 internals rounded once
     to fp32 (at g = 128 the scaled skew matrix is held in fp32): max-abs error and
     orthogonality |G^T G - I| within 1e-5 at every g (1e-6 / 4e-6 for g <= 64), including
-    a g = 128 set whose norm needs several squarings and g = 96 (padded to 128)."""
+    a g = 128 set whose norm needs several squarings, g = 96 (padded to 128) and g = 12 and
+    36 (padded to the next multiple of 8 for the fp64 tensor-core products)."""
     need_gpu()
     for g, sigma, n, tol, otol in [(8, 0.1, 64, 1e-6, 4e-6), (16, 0.1, 512, 1e-6, 4e-6), (32, 0.1, 64, 1e-6, 4e-6),
+                                   (12, 0.1, 32, 1e-6, 4e-6), (36, 0.05, 8, 1e-6, 4e-6),
                                    (64, 0.05, 16, 1e-6, 4e-6), (128, 0.05, 16, 1e-5, 1e-5), (128, 0.5, 4, 1e-5, 1e-5),
                                    (96, 0.05, 4, 1e-5, 1e-5)]:
         A = torch.randn(n, g, g, generator=torch.Generator().manual_seed(g)) * sigma

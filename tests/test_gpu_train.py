@@ -17,7 +17,7 @@ from tests.gpu_util import bf16_np, need_gpu
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("g", [8, 16, 32])
+@pytest.mark.parametrize("g", [6, 8, 16, 20, 32])
 def test_gauge_grad_matches_frechet_adjoint(g):
     need_gpu()
     rng = np.random.default_rng(g)
