@@ -242,6 +242,34 @@ cg_status cg_decode(const cg_kv_desc* kv, const cg_codec_desc* codec,
                     const uint8_t* codes_dev, const void* scales_dev, const void* zeros_dev,
                     const float* G_dev, int32_t t0, int32_t nt, void* kv_out_dev, void* stream);
 
+/* Workspace bytes cg_roundtrip_host needs: four layer-sized bf16 buffers,
+ * 4 * 2 B H T d * 2 bytes (host only). */
+cg_status cg_roundtrip_workspace_size(const cg_kv_desc* kv, uint64_t* bytes);
+
+/* cg_encode followed by cg_decode of the whole cache, with the cache and the
+ * decoded result in HOST memory (Codec-Gauge, Method: the codec round trip,
+ * with the recovery charged in timing).  The work is cut into layers: the copy
+ * of layer l + 1 to the device, the encode and decode of layer l and the copy
+ * of layer l - 1 back to the host run at the same time, on three internal
+ * non-blocking streams of the current device (created on first use and kept
+ * for the life of the process), so the two PCIe directions overlap each other
+ * and the kernels.
+ *   kv_host     bf16 [L][2][B][H][T][d] in host memory (input; page-locked
+ *               memory is needed for the copies to overlap)
+ *   G_dev, codes_dev, scales_dev, zeros_dev: as in cg_encode (the codes of the
+ *               whole cache are written, as by cg_encode over [0, T))
+ *   out_host    bf16 [L][2][B][H][T][d] in host memory (output: the decoded
+ *               cache, as cg_decode writes it)
+ *   workspace_dev / workspace_bytes: at least cg_roundtrip_workspace_size().
+ * The call is ordered after earlier work on `stream`, and later work on
+ * `stream` is ordered after all of it; the host buffers must stay valid and
+ * unchanged until then.  Argument errors as in cg_encode; CG_ERR_UNSUPPORTED
+ * when one layer's codes, steps or zero points are not a multiple of 16 bytes
+ * (the per-layer pointers must stay aligned). */
+cg_status cg_roundtrip_host(const cg_kv_desc* kv, const cg_codec_desc* codec, const void* kv_host,
+                            const float* G_dev, uint8_t* codes_dev, void* scales_dev, void* zeros_dev,
+                            void* out_host, void* workspace_dev, uint64_t workspace_bytes, void* stream);
+
 /* Decode-step attention settings.
  *   q_heads   query heads Hq, a multiple of the cache's KV heads H with
  *             Hq / H in {1, 2, 4, 8}; query head j uses KV head j / (Hq / H)

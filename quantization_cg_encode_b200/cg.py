@@ -20,7 +20,8 @@ ENGINE_AUTO, ENGINE_CUDA_CORES, ENGINE_CHAIN_TENSOR = 0, 1, 2
 
 # Every symbol include/cg.h declares.
 EXPORTS = ("cg_sizes_for", "cg_gauge_build", "cg_gauge_grad", "cg_adamw_step", "cg_group_gram", "cg_encode",
-           "cg_decode", "cg_decode_attention_workspace_size", "cg_decode_attention", "cg_spectral_workspace_size",
+           "cg_decode", "cg_roundtrip_workspace_size", "cg_roundtrip_host", "cg_decode_attention_workspace_size",
+           "cg_decode_attention", "cg_spectral_workspace_size",
            "cg_spectral_stats", "cg_spectral_stats_noalloc", "cg_selftest_wait_timeout", "cg_sync_status",
            "cg_last_cuda_error", "cg_status_string", "cg_version")
 
@@ -88,6 +89,9 @@ def lib():
         L.cg_group_gram.argtypes = [ctypes.POINTER(KvDesc), i32, vp, i32, i32, vp, vp]
         L.cg_encode.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, i32, i32, vp, vp, vp, vp, vp]
         L.cg_decode.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, vp, vp, i32, i32, vp, vp]
+        L.cg_roundtrip_workspace_size.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(ctypes.c_uint64)]
+        L.cg_roundtrip_host.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), vp, vp, vp, vp, vp, vp, vp,
+                                        ctypes.c_uint64, vp]
         L.cg_decode_attention_workspace_size.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(AttnDesc),
                                                          ctypes.POINTER(u64)]
         L.cg_decode_attention.argtypes = [ctypes.POINTER(KvDesc), ctypes.POINTER(CodecDesc), ctypes.POINTER(AttnDesc),
@@ -232,6 +236,39 @@ def cg_decode(kvd, codec, codes, scales, zeros, G, t0, nt, kv_out, stream=None):
                            _ptr(scales, torch.float16, "scales", sc), _ptr(zeros, torch.float16, "zeros", sc),
                            _ptr(G, torch.float32, "G", gauge_numel(kvd, codec.g)), int(t0), int(nt), _ptr(kv_out, torch.bfloat16, "kv_out", n),
                            _stream(stream)), "cg_decode")
+
+
+def cg_roundtrip_workspace_size(kvd):
+    out = ctypes.c_uint64()
+    _check(lib().cg_roundtrip_workspace_size(ctypes.byref(kvd), ctypes.byref(out)), "cg_roundtrip_workspace_size")
+    return int(out.value)
+
+
+def _host_ptr(t, dtype, name, numel):
+    """Host pointer of a contiguous CPU tensor of the given dtype."""
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError("%s must be a CPU tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.numel() < numel:
+        raise ValueError("%s holds %d elements, needs %d" % (name, t.numel(), numel))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def cg_roundtrip_host(kvd, codec, kv_host, G, codes, scales, zeros, out_host, workspace, stream=None):
+    """Encode a host-resident cache (bf16 CPU tensor, pinned for overlap) into device codes and
+    decode it back into out_host, pipelined by layer."""
+    n = kvd.layers * 2 * kvd.batch * kvd.heads * kvd.tokens * kvd.d_head
+    cb, sc = cg_sizes_for(kvd, codec)
+    _check(lib().cg_roundtrip_host(ctypes.byref(kvd), ctypes.byref(codec), _host_ptr(kv_host, torch.bfloat16, "kv_host", n),
+                                   _ptr(G, torch.float32, "G", gauge_numel(kvd, codec.g)),
+                                   _ptr(codes, torch.uint8, "codes", cb), _ptr(scales, torch.float16, "scales", sc),
+                                   _ptr(zeros, torch.float16, "zeros", sc),
+                                   _host_ptr(out_host, torch.bfloat16, "out_host", n),
+                                   _ptr(workspace, torch.uint8, "workspace"),
+                                   workspace.numel(), _stream(stream)), "cg_roundtrip_host")
 
 
 def attn_desc(q_heads, n_tokens, layer0=0, n_layers=1, scale=None, d_head=128):

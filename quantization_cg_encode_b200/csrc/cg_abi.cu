@@ -11,10 +11,12 @@ __device__ unsigned int g_status = 0;
 using namespace cg;
 
 namespace {
+bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 6 || b == 8; }
+}  // namespace
+
+namespace cg {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
-
-bool valid_bits(int b) { return b == 2 || b == 3 || b == 4 || b == 6 || b == 8; }
 
 cg_status check_kv(const cg_kv_desc* kv) {
   if (!kv) return CG_ERR_INVALID;
@@ -50,6 +52,10 @@ cg_status check_codec(const cg_kv_desc* kv, const cg_codec_desc* c) {
     return CG_ERR_UNSUPPORTED;
   return CG_OK;
 }
+
+}  // namespace cg
+
+namespace {
 
 cg_status check_range(const cg_kv_desc* kv, const cg_codec_desc* c, int t0, int nt) {
   const int step = c->mode == CG_QUANT_KIVI ? 32 : c->tb;

@@ -52,6 +52,10 @@ cudaError_t launch_spectral_generic(const KvGeom& k, int x_fp32, const void* x, 
 // for cg_last_cuda_error), shared by the entry points.
 int num_sms();
 cg_status from_cuda(cudaError_t e);
+// Host validation shared by the entry points: 16-byte alignment, the cache shape, the codec.
+bool aligned16(const void* p);
+cg_status check_kv(const cg_kv_desc* kv);
+cg_status check_codec(const cg_kv_desc* kv, const cg_codec_desc* c);
 cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f, float lambda_r,
                             float tau, float* lfreq, float* lrate, double* totals, float* dG, void* workspace,
                             unsigned int* status, int num_sms, cudaStream_t st);

@@ -123,3 +123,25 @@ def test_attention_validation_without_gpu():
              cg.CG_ERR_INVALID]
     for at, want in zip(bad, codes):
         assert L.cg_decode_attention_workspace_size(ctypes.byref(kvd), ctypes.byref(at), ctypes.byref(out)) == want
+
+
+def _rt(kvd, codec, kv=0x10000, G=0x20000, codes=0x30000, sc=0x40000, z=0x50000, out=0x60000, ws=0x70000,
+        ws_bytes=1 << 40):
+    L = cg.lib()
+    vp = ctypes.c_void_p
+    return L.cg_roundtrip_host(ctypes.byref(kvd), ctypes.byref(codec), vp(kv), vp(G), vp(codes), vp(sc), vp(z),
+                               vp(out), vp(ws), ws_bytes, None)
+
+
+def test_roundtrip_workspace_and_validation_without_gpu():
+    kvd = cg.kv_desc(32, 1, 8, 4096, 128)
+    assert cg.cg_roundtrip_workspace_size(kvd) == 4 * 2 * 8 * 4096 * 128 * 2   # four one-layer bf16 buffers
+    ok = cg.codec_desc(g=16, bits=4)
+    assert _rt(kvd, ok, kv=0) == cg.CG_ERR_INVALID                        # null host input
+    assert _rt(kvd, ok, out=0) == cg.CG_ERR_INVALID                       # null host output
+    assert _rt(kvd, ok, codes=0x30008) == cg.CG_ERR_INVALID               # misaligned device output
+    assert _rt(kvd, ok, ws=0x70004) == cg.CG_ERR_INVALID                  # misaligned workspace
+    assert _rt(kvd, ok, ws_bytes=cg.cg_roundtrip_workspace_size(kvd) - 16) == cg.CG_ERR_INVALID
+    assert _rt(kvd, cg.codec_desc(g=16, bits=5)) == cg.CG_ERR_UNSUPPORTED
+    # one layer's steps with 16 x d ranges: 2 B H (T / 16) fp16 = 8 bytes here, not a multiple of 16
+    assert _rt(cg.kv_desc(2, 1, 1, 32, 64), cg.codec_desc(g=16, bits=4, range_cols=64)) == cg.CG_ERR_UNSUPPORTED
