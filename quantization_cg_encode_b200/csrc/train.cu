@@ -41,45 +41,92 @@ cudaError_t launch_adamw(float* p, const float* grad, float* m, float* v, long l
 }
 
 namespace {
-constexpr int kGramThreads = 256;
+constexpr int kGramThreads = 256, kGramWarps = kGramThreads / 32;
 constexpr int kGramTok = 32;  // tokens staged per step
 }  // namespace
 
 // One thread block per gauge set (l, s, h): sums over the batch and tokens
-// [t0, t0 + nt) in order; thread e owns entries e + 256 k of [R][g][g].
+// [t0, t0 + nt) in a fixed order, on the fp64 tensor cores.  C_r = X_r^T X_r is
+// cut into 8 x 8 tiles (i block, j block) of every group r; warp w owns tiles
+// w, w + 8, .. and accumulates each with mma.sync m8n8k4 fp64 over 4 tokens per
+// step (A = X_r^T: row lane / 4, column lane % 4; B = X_r: row lane % 4, column
+// lane / 4; C row lane / 4, columns 2 (lane % 4) + {0, 1}).  bf16 inputs are
+// exact in fp64, so every product is exact; a staged step's missing tokens are
+// zeros.  The row pitch D + 8 (floats) puts the 4 token rows of a fragment on
+// disjoint banks.
 template <int D, int G>
-__global__ void __launch_bounds__(kGramThreads) gram_kernel(const uint16_t* __restrict__ kv, double* __restrict__ gram,
-                                                            KvGeom k, int t0, int nt) {
-  constexpr int R = D / G;
-  constexpr int PER = R * G * G / kGramThreads;  // entries per thread
-  static_assert(PER * kGramThreads == R * G * G, "entries divide evenly");
-  __shared__ float xs[kGramTok][D + 1];
+__global__ void __launch_bounds__(kGramThreads, 1) gram_kernel(const uint16_t* __restrict__ kv, double* __restrict__ gram,
+                                                               KvGeom k, int t0, int nt) {
+  constexpr int R = D / G, TN = G / 8, TILES = R * TN * TN, PER = TILES / kGramWarps, P = D + 8;
+  constexpr int VEC = kGramTok * D / 8 / kGramThreads;  // 16-byte loads per thread per staged step
+  static_assert(PER * kGramWarps == TILES, "tiles divide evenly");
+  static_assert(VEC * 8 * kGramThreads == kGramTok * D, "loads divide evenly");
+  __shared__ __align__(16) float xs[2][kGramTok][P];
   const int set = blockIdx.x;  // (l * 2 + s) * H + h
   const int h = set % k.H, ls = set / k.H;
-  double acc[PER];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, lr = lane >> 2, lc = lane & 3;
+  int ca[PER], cb[PER];  // fragment columns of this lane: channel of A (row block) and of B (column block)
 #pragma unroll
-  for (int q = 0; q < PER; ++q) acc[q] = 0.0;
-  for (int b = 0; b < k.B; ++b) {
+  for (int q = 0; q < PER; ++q) {
+    const int t = warp + kGramWarps * q, r = t / (TN * TN), ti = (t / TN) % TN, tj = t % TN;
+    ca[q] = r * G + 8 * ti + lr;
+    cb[q] = r * G + 8 * tj + lr;
+  }
+  double acc[PER][2];
+#pragma unroll
+  for (int q = 0; q < PER; ++q) acc[q][0] = acc[q][1] = 0.0;
+  // staged steps: (batch b, 32 tokens from t0 + 32 j), in order; missing tokens read as zeros
+  const int nch = (nt + kGramTok - 1) / kGramTok, total = k.B * nch;
+  auto fetch = [&](int ci, uint4 (&v)[VEC]) {
+    const int b = ci / nch, tt = (ci % nch) * kGramTok, ntok = min(kGramTok, nt - tt);
     const long long slice = ((long long)ls * k.B + b) * k.H + h;
-    const uint16_t* x = kv + (slice * k.T + t0) * D;
-    for (int tt = 0; tt < nt; tt += kGramTok) {
-      const int ntok = min(kGramTok, nt - tt);
-      __syncthreads();
-      for (int e = threadIdx.x; e < ntok * D; e += kGramThreads)
-        xs[e / D][e % D] = bf16lo((uint32_t)x[(long long)tt * D + e]);
-      __syncthreads();
+    const uint16_t* x = kv + (slice * k.T + t0 + tt) * D;
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) {
+      const int e = threadIdx.x + kGramThreads * j, t = e / (D / 8), c8 = e % (D / 8);
+      v[j] = t < ntok ? __ldg(reinterpret_cast<const uint4*>(x + (long long)t * D) + c8) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto stage = [&](const uint4 (&v)[VEC], int buf) {
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) {
+      const int e = threadIdx.x + kGramThreads * j, t = e / (D / 8), c8 = e % (D / 8);
+      float4* dst = reinterpret_cast<float4*>(&xs[buf][t][8 * c8]);
+      dst[0] = make_float4(bf16lo(v[j].x), bf16hi(v[j].x), bf16lo(v[j].y), bf16hi(v[j].y));
+      dst[1] = make_float4(bf16lo(v[j].z), bf16hi(v[j].z), bf16lo(v[j].w), bf16hi(v[j].w));
+    }
+  };
+  if (total > 0) {
+    uint4 v[VEC];
+    fetch(0, v);
+    stage(v, 0);
+  }
+  __syncthreads();
+  for (int ci = 0; ci < total; ++ci) {
+    uint4 v[VEC];
+    if (ci + 1 < total) fetch(ci + 1, v);  // the next step's loads are in flight during this one
+    const int tt = (ci % nch) * kGramTok, steps = (min(kGramTok, nt - tt) + 3) >> 2;
+    for (int s4 = 0; s4 < steps; ++s4) {
+      const float* row = xs[ci & 1][4 * s4 + lc];
 #pragma unroll
       for (int q = 0; q < PER; ++q) {
-        const int e = threadIdx.x + kGramThreads * q;
-        const int r = e / (G * G), i = (e / G) % G, j = e % G;
-        double a = acc[q];
-        for (int t = 0; t < ntok; ++t) a = fma((double)xs[t][r * G + i], (double)xs[t][r * G + j], a);
-        acc[q] = a;
+        const double a = (double)row[ca[q]], bb = (double)row[cb[q]];
+        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                     : "+d"(acc[q][0]), "+d"(acc[q][1])
+                     : "d"(a), "d"(bb));
       }
     }
+    if (ci + 1 < total) stage(v, (ci + 1) & 1);
+    __syncthreads();
   }
+  double* out = gram + (long long)set * R * G * G;
 #pragma unroll
-  for (int q = 0; q < PER; ++q) gram[(long long)set * R * G * G + threadIdx.x + kGramThreads * q] = acc[q];
+  for (int q = 0; q < PER; ++q) {
+    const int t = warp + kGramWarps * q, r = t / (TN * TN), ti = (t / TN) % TN, tj = t % TN;
+    double* o = out + (r * G + 8 * ti + lr) * G + 8 * tj + 2 * lc;
+    o[0] = acc[q][0];
+    o[1] = acc[q][1];
+  }
 }
 
 cudaError_t launch_gram(const KvGeom& k, int g, const uint16_t* kv, double* gram, int t0, int nt, cudaStream_t st) {
