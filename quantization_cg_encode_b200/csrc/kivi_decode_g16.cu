@@ -12,16 +12,20 @@
 //   * values: the step and zero point are one per token, so
 //       x_hat_n = s_t sum_c q_c G[c][n] + z_t colsum_n
 //     with the codes themselves as the A operand (integers, exact in fp16);
-//   * keys: the step and zero point vary with the channel, so A is the
-//     dequantized y = s_c q + z_c (fp32), split into fp16 hi + lo, and
-//       x_hat = A_hi G_hi + A_hi G_lo + A_lo G_hi
-//     (a unit whose |y| could leave the fp16 range is scaled by a power of
-//     two, exactly undone afterwards).
+//   * keys: the step and zero point vary with the channel (and are fixed
+//     over the unit's 32 tokens), so the step moves into the gauge:
+//       x_hat_n = sum_c q_c (s_c G[c][n]) + sum_c z_c G[c][n],
+//     with the codes again as the A operand, G'[c][n] = 2^e s_c G[c][n] split
+//     into fp16 hi + lo once per unit (2^e a power of two that puts the largest
+//     step near 2^13, undone exactly afterwards) and the second sum, a vector
+//     per unit, added in the epilogue.
 // The k order of A and B is permuted consistently (each thread reads 4
-// adjacent channels).  Each bf16 16-token tile goes through a padded shared-
-// memory staging with stmatrix and leaves with full-line 16-byte stores.  The
-// per-warp buffers are sized by the code width, so that two CTAs (16 warps)
-// share an SM at every code width.
+// adjacent channels), and so are the MMA rows: row g4 (+ 8) of 16-token tile
+// tt is token 4 g4 + 2 tt (+ 1) of the unit, so a thread's tokens are four
+// consecutive ones and each key record yields them in one read.  Each bf16
+// 16-token tile goes through a padded shared-memory staging with stmatrix and
+// leaves with full-line 16-byte stores.  The per-warp buffers are sized by the
+// code width, so that two CTAs (16 warps) share an SM at every code width.
 #include "cg_kernels.cuh"
 
 namespace cg {
@@ -54,14 +58,6 @@ __device__ __forceinline__ uint32_t f16pair(uint32_t c_lo, uint32_t c_hi) {
   return f16_sub1024(0x64006400u | c_lo | (c_hi << 16));
 }
 __device__ __forceinline__ uint32_t f16_bits(float x) { return (uint32_t)__half_as_ushort(__float2half_rn(x)); }
-// fp16 hi and lo words of two fp32 values: hi = fp16(v), lo = fp16(v - hi)
-__device__ __forceinline__ void f16_split2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
-  const __half2 h = __floats2half2_rn(v0, v1);
-  const float2 hf = __half22float2(h);
-  const __half2 l = __floats2half2_rn(v0 - hf.x, v1 - hf.y);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = *reinterpret_cast<const uint32_t*>(&l);
-}
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)), "l"(gmem)
                : "memory");
@@ -140,7 +136,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) kivi_decode_g16_kernel(CodecAr
     int l, sk, b, h;
     slice_coords(slice, a.k, l, sk, b, h);
     const bool key = sk == 0;
-    if (slice != loaded) {  // G fragments and column sums of this head slice
+    if (!key && slice != loaded) {  // values: G fragments and column sums of this head slice
       const float* G0 = a.G + gauge_set(l, sk, h, a.k) * NG * 256;
 #pragma unroll
       for (int r = 0; r < NG; ++r) {
@@ -173,22 +169,60 @@ __global__ void __launch_bounds__(kWarps * 32, 2) kivi_decode_g16_kernel(CodecAr
       }
       loaded = slice;
     }
-    // keys: a power of two that keeps every |y| of the unit inside fp16
-    float kscale = 1.0f, kunscale = 1.0f;
+    // keys: G' = 2^e s_c G per unit (fp16 hi + lo) and the bias sum_c z_c G[c][n] in csum
+    float kunscale = 1.0f;
     if (key) {
-      float big = 0.0f;
+      float smax = 0.0f;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int c = 4 * lane + m;
-        const float s = __half2float(__ushort_as_half(sbuf[c])), z = __half2float(__ushort_as_half(zbuf[c]));
-        big = fmaxf(big, fabsf(z) + s * (float)M);
+      for (int m = 0; m < 4; ++m) smax = fmaxf(smax, __half2float(__ushort_as_half(sbuf[4 * lane + m])));
+      smax = warp_max_f32(smax);
+      float kscale = 1.0f;
+      if (smax > 0.0f) {  // smax in [2^x, 2^(x+1)): scale 2^(13 - x), exact both ways (x in [-24, 15])
+        const int x = (int)((__float_as_uint(smax) >> 23) & 0xffu) - 127;
+        kscale = __uint_as_float((uint32_t)(127 + 13 - x) << 23);
+        kunscale = __uint_as_float((uint32_t)(127 - 13 + x) << 23);
       }
-      big = warp_max_f32(big);
-      // warp-uniform, exact powers of two; finite fp16 steps and zero points need at most 3 steps
-      for (int it = 0; it < 8 && big * kscale > 16384.0f; ++it) {
-        kscale *= 0.0625f;
-        kunscale *= 16.0f;
+      const float* G0 = a.G + gauge_set(l, sk, h, a.k) * NG * 256;
+#pragma unroll
+      for (int r = 0; r < NG; ++r) {
+        float sc[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) sc[m] = __half2float(__ushort_as_half(sbuf[16 * r + 4 * q4 + m])) * kscale;
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+          const float* Gc = G0 + r * 256 + (4 * q4) * 16 + 8 * nh + g4;
+          float hi[4], lo[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const float v = __ldg(Gc + m * 16) * sc[m];
+            hi[m] = __half2float(__float2half_rn(v));
+            lo[m] = v - hi[m];
+          }
+          const __half2 h01 = __floats2half2_rn(hi[0], hi[1]), h23 = __floats2half2_rn(hi[2], hi[3]);
+          const __half2 l01 = __floats2half2_rn(lo[0], lo[1]), l23 = __floats2half2_rn(lo[2], lo[3]);
+          bfr[r][nh][0][0] = *reinterpret_cast<const uint32_t*>(&h01);
+          bfr[r][nh][0][1] = *reinterpret_cast<const uint32_t*>(&h23);
+          bfr[r][nh][1][0] = *reinterpret_cast<const uint32_t*>(&l01);
+          bfr[r][nh][1][1] = *reinterpret_cast<const uint32_t*>(&l23);
+        }
       }
+      {  // bias of channels n = 4 lane .. 4 lane + 3 (group lane / 4)
+        const int rg = lane >> 2, n0 = 4 * (lane & 3);
+        float4 bsum = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float z = __half2float(__ushort_as_half(zbuf[16 * rg + i]));
+          const float4 gv = __ldg(reinterpret_cast<const float4*>(G0 + rg * 256 + i * 16 + n0));
+          bsum.x = __fmaf_rn(z, gv.x, bsum.x);
+          bsum.y = __fmaf_rn(z, gv.y, bsum.y);
+          bsum.z = __fmaf_rn(z, gv.z, bsum.z);
+          bsum.w = __fmaf_rn(z, gv.w, bsum.w);
+        }
+        __syncwarp();  // the previous unit's epilogue has read csum
+        *reinterpret_cast<float4*>(csum + 4 * lane) = bsum;
+        __syncwarp();
+      }
+      loaded = -1;  // csum now holds a key bias: a later value slice rebuilds its column sums
     }
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
@@ -201,7 +235,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) kivi_decode_g16_kernel(CodecAr
           float sv[2], zv[2];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            const int t = 16 * tt + g4 + 8 * half;
+            const int t = 4 * g4 + 2 * tt + half;  // MMA row g4 + 8 half of tile tt
             const int bit = ((t * 4 + (r >> 1)) * 32 + 16 * (r & 1) + 4 * q4) * BITS;
             const uint32_t v = bits_at(cbuf, bit);
             const uint32_t c0 = v & M, c1 = (v >> BITS) & M, c2 = (v >> (2 * BITS)) & M, c3 = (v >> (3 * BITS)) & M;
@@ -221,48 +255,39 @@ __global__ void __launch_bounds__(kWarps * 32, 2) kivi_decode_g16_kernel(CodecAr
             pk[nh][1] = pack_bf16x2(__fmaf_rn(sv[1], acc[2], zv[1] * cs2.x), __fmaf_rn(sv[1], acc[3], zv[1] * cs2.y));
           }
         } else {
-          // keys: record (channel c) holds the unit's 32 tokens; y = s_c q + z_c
-          float sc[4], zc[4];
+          // keys: record (channel c) holds the unit's 32 tokens; this thread's tokens
+          // 4 g4 .. 4 g4 + 3 of channel 16 r + 4 q4 + m are 4 BITS consecutive bits
+          uint32_t w[4];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int c = 16 * r + 4 * q4 + m;
-            sc[m] = __half2float(__ushort_as_half(sbuf[c])) * kscale;
-            zc[m] = __half2float(__ushort_as_half(zbuf[c])) * kscale;
-          }
-          uint32_t ahi[4], alo[4];
+          for (int m = 0; m < 4; ++m) w[m] = bits_at(cbuf, (16 * r + 4 * q4 + m) * 32 * BITS + 4 * g4 * BITS);
+          uint32_t afr[4];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            const int t = 16 * tt + g4 + 8 * half;
-            float y[4];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const int c = 16 * r + 4 * q4 + m;
-              const uint32_t q = bits_at(cbuf, c * 32 * BITS + t * BITS) & M;
-              y[m] = __fmaf_rn(sc[m], (float)q, zc[m]);
-            }
-            f16_split2(y[0], y[1], ahi[half], alo[half]);
-            f16_split2(y[2], y[3], ahi[2 + half], alo[2 + half]);
+            const int sh = (2 * tt + half) * BITS;
+            afr[half] = f16pair((w[0] >> sh) & M, (w[1] >> sh) & M);
+            afr[2 + half] = f16pair((w[2] >> sh) & M, (w[3] >> sh) & M);
           }
 #pragma unroll
           for (int nh = 0; nh < 2; ++nh) {
             float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            mma_f16(acc, alo, bfr[r][nh][0][0], bfr[r][nh][0][1]);
-            mma_f16(acc, ahi, bfr[r][nh][1][0], bfr[r][nh][1][1]);
-            mma_f16(acc, ahi, bfr[r][nh][0][0], bfr[r][nh][0][1]);
-            pk[nh][0] = pack_bf16x2(acc[0] * kunscale, acc[1] * kunscale);
-            pk[nh][1] = pack_bf16x2(acc[2] * kunscale, acc[3] * kunscale);
+            mma_f16(acc, afr, bfr[r][nh][1][0], bfr[r][nh][1][1]);
+            mma_f16(acc, afr, bfr[r][nh][0][0], bfr[r][nh][0][1]);
+            const float2 b2 = *reinterpret_cast<const float2*>(csum + 16 * r + 8 * nh + 2 * q4);
+            pk[nh][0] = pack_bf16x2(__fmaf_rn(acc[0], kunscale, b2.x), __fmaf_rn(acc[1], kunscale, b2.y));
+            pk[nh][1] = pack_bf16x2(__fmaf_rn(acc[2], kunscale, b2.x), __fmaf_rn(acc[3], kunscale, b2.y));
           }
         }
         // tiles (rows 0-7 | 8-15 of this 16-token tile) x (cols 16r .. +7 | 16r+8 .. +15)
         stmatrix_x4(st_addr + 32 * r, pk[0][0], pk[0][1], pk[1][0], pk[1][1]);
       }
       __syncwarp();
-      // the tile's 16 rows of 256 B, contiguous in the output: each instruction writes two whole rows
-      uint16_t* obase = a.kv_out + (slice * a.k.T + 32LL * tgroup + 16 * tt) * D;
+      // the tile's 16 rows of 256 B (row g + 8 h is token 4 g + 2 tt + h): each instruction writes two whole rows
+      uint16_t* obase = a.kv_out + (slice * a.k.T + 32LL * tgroup) * D;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int row = 2 * k + (lane >> 4), ch = lane & 15;
-        reinterpret_cast<uint4*>(obase + row * D)[ch] = *reinterpret_cast<const uint4*>(stg + row * kPitch + ch * 16);
+        const int tok = 4 * (row & 7) + 2 * tt + (row >> 3);
+        reinterpret_cast<uint4*>(obase + tok * D)[ch] = *reinterpret_cast<const uint4*>(stg + row * kPitch + ch * 16);
       }
       __syncwarp();
     }
