@@ -349,10 +349,12 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
 namespace {
 constexpr int kDecEpi = 8;  // two warpgroups taking alternate blocks: code expansion, then epilogue
 constexpr int kDecThreads = (kDecEpi + 2) * 32;
+constexpr int kStgPitch = 256 + 16, kStgWarp = 32 * kStgPitch;
 struct FdSmem {
   unsigned char* as;  // 2 x 32 KB A tiles
   unsigned char* gs;  // 2 x 32 KB G^T tiles
   float* colsum;      // 2 x 128
+  unsigned char* stg; // per epilogue warp: 32 output rows of 256 B (+16 B pad) for coalesced stores
   uint64_t* a_full;
   uint64_t* a_empty;
   uint64_t* g_full;
@@ -367,7 +369,8 @@ __device__ inline FdSmem fd_carve(unsigned char* raw) {
   s.as = base;
   s.gs = base + 2 * kBlockBytes;
   s.colsum = reinterpret_cast<float*>(base + 4 * kBlockBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.colsum + 256);
+  s.stg = reinterpret_cast<unsigned char*>(s.colsum + 256);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.stg + kDecEpi * kStgWarp);
   s.a_full = bars;
   s.a_empty = bars + 2;
   s.g_full = bars + 4;
@@ -377,7 +380,7 @@ __device__ inline FdSmem fd_carve(unsigned char* raw) {
   s.tmem_base = reinterpret_cast<uint32_t*>(bars + 12);
   return s;
 }
-constexpr int kFdSmem = 1024 + 4 * kBlockBytes + 256 * 4 + 12 * 8 + 16;
+constexpr int kFdSmem = 1024 + 4 * kBlockBytes + 256 * 4 + kDecEpi * kStgWarp + 12 * 8 + 16;
 
 // bf16 bits of two codes (< 256, exact), packed low / high
 __device__ __forceinline__ uint32_t code_pair_bf16(uint32_t q0, uint32_t q1) {
@@ -575,27 +578,56 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
         tc_fence_after();
         const uint32_t taddr = tmem + ab * 128 + ((uint32_t)(32 * quarter) << 16);
         const float* cs = sm.colsum + gb * 128;
-        uint4* dst = reinterpret_cast<uint4*>(a.kv_out + (slice * a.k.T + tok) * (long long)D);
+        unsigned char* stg = sm.stg + warp * kStgWarp;
+        // 32 accumulator columns c4 -> 64 bytes of this thread's staged row
+        auto emit = [&](const float (&v)[32], int c4) {
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float v[32];
-          tmem_ld32(taddr + 32 * c4, v);
-          tmem_wait_ld();
-          if (row < valid) {
-#pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              uint4 o;
-              o.x = pack_bf16x2(__fmaf_rn(sf, v[j + 0], zf * cs[32 * c4 + j + 0]), __fmaf_rn(sf, v[j + 1], zf * cs[32 * c4 + j + 1]));
-              o.y = pack_bf16x2(__fmaf_rn(sf, v[j + 2], zf * cs[32 * c4 + j + 2]), __fmaf_rn(sf, v[j + 3], zf * cs[32 * c4 + j + 3]));
-              o.z = pack_bf16x2(__fmaf_rn(sf, v[j + 4], zf * cs[32 * c4 + j + 4]), __fmaf_rn(sf, v[j + 5], zf * cs[32 * c4 + j + 5]));
-              o.w = pack_bf16x2(__fmaf_rn(sf, v[j + 6], zf * cs[32 * c4 + j + 6]), __fmaf_rn(sf, v[j + 7], zf * cs[32 * c4 + j + 7]));
-              dst[(32 * c4 + j) / 8] = o;
-            }
+          for (int j = 0; j < 32; j += 8) {
+            uint4 o;
+            o.x = pack_bf16x2(__fmaf_rn(sf, v[j + 0], zf * cs[32 * c4 + j + 0]), __fmaf_rn(sf, v[j + 1], zf * cs[32 * c4 + j + 1]));
+            o.y = pack_bf16x2(__fmaf_rn(sf, v[j + 2], zf * cs[32 * c4 + j + 2]), __fmaf_rn(sf, v[j + 3], zf * cs[32 * c4 + j + 3]));
+            o.z = pack_bf16x2(__fmaf_rn(sf, v[j + 4], zf * cs[32 * c4 + j + 4]), __fmaf_rn(sf, v[j + 5], zf * cs[32 * c4 + j + 5]));
+            o.w = pack_bf16x2(__fmaf_rn(sf, v[j + 6], zf * cs[32 * c4 + j + 6]), __fmaf_rn(sf, v[j + 7], zf * cs[32 * c4 + j + 7]));
+            *reinterpret_cast<uint4*>(stg + lane * kStgPitch + 2 * (32 * c4 + j)) = o;
           }
-        }
+        };
+        // two 32-column loads in flight: the next one is issued before the current one is used
+        // (the empty asm statements pin each load's registers after its wait)
+        float va[32], vb[32];
+        tmem_ld32(taddr, va);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) asm volatile("" : "+f"(va[k]));
+        tmem_ld32(taddr + 32, vb);
+        emit(va, 0);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) asm volatile("" : "+f"(vb[k]));
+        tmem_ld32(taddr + 64, va);
+        emit(vb, 1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) asm volatile("" : "+f"(va[k]));
+        tmem_ld32(taddr + 96, vb);
+        emit(va, 2);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) asm volatile("" : "+f"(vb[k]));
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.t_empty[ab]);
+        if (lane == 0) mbar_arrive(&sm.t_empty[ab]);  // the accumulator is in registers
+        emit(vb, 3);
+        __syncwarp();
+        // the warp's 32 rows leave as whole 256-byte lines: two rows per instruction
+        const int tok0 = a.t0 + 128 * bq + 32 * quarter;
+        uint4* dst0 = reinterpret_cast<uint4*>(a.kv_out + (slice * a.k.T + tok0) * (long long)D);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int r = 2 * k + (lane >> 4), ch = lane & 15;
+          if (32 * quarter + r < valid)
+            dst0[r * (D / 8) + ch] = *reinterpret_cast<const uint4*>(stg + r * kStgPitch + 16 * ch);
+        }
+        __syncwarp();  // the staging rows are rewritten by this warp's next block
       }
       if (last_of_slice) {  // every epilogue warp is past this slice: its G^T and column sums may go
         __syncwarp();
