@@ -261,41 +261,56 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
         const uint32_t taddr = tmem + acc * 128 + ((uint32_t)(32 * quarter) << 16);
         const int valid = min(128, a.nt - 128 * bq);
         const int tok = a.t0 + 128 * bq + row;
+        // Two 32-column accumulator loads are kept in flight in both passes: the next one is
+        // issued before the current one is used (the empty asm statements pin each load's
+        // registers after its wait).
+        float va[32], vb[32];
+        auto pin = [](float (&v)[32]) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) asm volatile("" : "+f"(v[k]));
+        };
         // pass 1: the row's range, then the 16-token block's (16 lanes)
         float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(taddr + 32 * c, v);
-          tmem_wait_ld();
+        auto range32 = [&](const float (&v)[32]) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            mn = fminf(mn, v[j]);
-            mx = fmaxf(mx, v[j]);
+          for (int j = 0; j < 32; j += 2) {
+            mn = min3f(mn, v[j], v[j + 1]);
+            mx = max3f(mx, v[j], v[j + 1]);
           }
-        }
+        };
+        tmem_ld32(taddr, va);
+        tmem_wait_ld();
+        pin(va);
+        tmem_ld32(taddr + 32, vb);
+        range32(va);
+        tmem_wait_ld();
+        pin(vb);
+        tmem_ld32(taddr + 64, va);
+        range32(vb);
+        tmem_wait_ld();
+        pin(va);
+        tmem_ld32(taddr + 96, vb);
+        range32(va);
+        tmem_wait_ld();
+        pin(vb);
+        range32(vb);
 #pragma unroll
         for (int o = 8; o >= 1; o >>= 1) {
           mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         }
         const QParams qp = quant_params(mn, mx, inv_qmax);
+        // t is monotone in y: no clamp is needed when the block's extremes round into [0, qmax]
+        const float t_lo = __fmul_rn(__fsub_rn(mn, qp.zf), qp.inv), t_hi = __fmul_rn(__fsub_rn(mx, qp.zf), qp.inv);
+        const bool clampit = !(t_lo >= -0.5f && t_hi < (float)QMAX + 0.5f);
+        const f2_t nz2 = f2_make(-qp.zf, -qp.zf), iv2 = f2_make(qp.inv, qp.inv), mg2 = f2_make(12582912.0f, 12582912.0f);
         // pass 2: codes of the row, 32 at a time (BITS packed words each, little-endian),
         // stored as they are made: the row's codes are bytes [r16 * 16 * BITS, +16 * BITS)
         // of its 16-token block's record
         const int tile = tok / 16, r16 = tok % 16;
         unsigned char* dst = a.codes + slice * slice_code_bytes + (long long)tile * (16 * D * BITS / 8) +
                              r16 * (D * BITS / 8);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float v[32];
-          tmem_ld32(taddr + 32 * c, v);
-          tmem_wait_ld();
-          if (c == 3) {  // the accumulator is free once the last columns are in registers
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.t_empty[acc]);
-          }
+        auto quant32 = [&](const float (&v)[32], int c) {
           if (a.gauged && row < valid) {
             float4* gd = reinterpret_cast<float4*>(a.gauged + (slice * a.k.T + tok) * D + 32 * c);
 #pragma unroll
@@ -305,17 +320,46 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
 #pragma unroll
           for (int w = 0; w < BITS; ++w) words[w] = 0;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            // q = clamp(rne(fl(fl(y - z) * inv)), 0, qmax): clamped first, then rounded (RNE)
-            // by adding 1.5 * 2^23, which leaves the integer in the low mantissa bits
-            const float t = fminf(fmaxf(__fmul_rn(__fsub_rn(v[j], qp.zf), qp.inv), 0.0f), (float)QMAX);
-            const uint32_t q = __float_as_uint(__fadd_rn(t, 12582912.0f)) & ((1u << BITS) - 1u);
-            const int bit = j * BITS;
-            words[bit >> 5] |= q << (bit & 31);
-            if ((bit & 31) + BITS > 32) words[(bit >> 5) + 1] |= q >> (32 - (bit & 31));
+          for (int j = 0; j < 32; j += 2) {
+            // q = clamp(rne(fl(fl(y - z) * inv)), 0, qmax): clamped where needed, then rounded
+            // (RNE) by adding 1.5 * 2^23, which leaves the integer in the low mantissa bits
+            float t0, t1;
+            f2_split(f2_mul(f2_add(f2_make(v[j], v[j + 1]), nz2), iv2), t0, t1);
+            if (clampit) {
+              t0 = fminf(fmaxf(t0, 0.0f), (float)QMAX);
+              t1 = fminf(fmaxf(t1, 0.0f), (float)QMAX);
+            }
+            float r0, r1;
+            f2_split(f2_add(f2_make(t0, t1), mg2), r0, r1);
+            const uint32_t q[2] = {__float_as_uint(r0) & (uint32_t)QMAX, __float_as_uint(r1) & (uint32_t)QMAX};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int bit = (j + e) * BITS;
+              words[bit >> 5] |= q[e] << (bit & 31);
+              if ((bit & 31) + BITS > 32) words[(bit >> 5) + 1] |= q[e] >> (32 - (bit & 31));
+            }
           }
           if (row < valid) store_code_words<BITS>(dst + c * 4 * BITS, words);
-        }
+        };
+        tmem_ld32(taddr, va);
+        tmem_wait_ld();
+        pin(va);
+        tmem_ld32(taddr + 32, vb);
+        quant32(va, 0);
+        tmem_wait_ld();
+        pin(vb);
+        tmem_ld32(taddr + 64, va);
+        quant32(vb, 1);
+        tmem_wait_ld();
+        pin(va);
+        tmem_ld32(taddr + 96, vb);
+        quant32(va, 2);
+        tmem_wait_ld();
+        pin(vb);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.t_empty[acc]);  // the accumulator is in registers
+        quant32(vb, 3);
         if (row < valid && (lane & 15) == 0) {
           const long long bidx = slice * (a.k.T / 16) + tile;
           a.scales[bidx] = qp.sh;
