@@ -50,7 +50,10 @@ typedef enum {
   CG_ERR_UNSUPPORTED = 2, /* valid request this build has no kernel for     */
   CG_ERR_CUDA = 3,        /* launch or runtime error                        */
   CG_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out             */
-  CG_ERR_TOO_LARGE = 5    /* request exceeds a fixed, built-in scratch size */
+  CG_ERR_TOO_LARGE = 5,   /* request exceeds a fixed, built-in scratch size */
+  CG_ERR_BOUND = 6        /* CG_ENGINE_CHAIN_TENSOR: a tensor-core value lay
+                             farther from the fp32 chain than the error bound
+                             its decisions assume (see cg_sync_status)      */
 } cg_status;
 
 typedef enum {
@@ -80,7 +83,12 @@ typedef enum {
                                  into three bf16 terms, and the chain re-evaluated
                                  wherever the tensor-core value could change a
                                  decision (needs G orthogonal to 2^-12, checked
-                                 per head slice; else the chain throughout) */
+                                 per head slice; else the chain throughout).
+                                 The decisions assume a tensor-core accumulation
+                                 error of at most 2^-20 sum_j |G_ij x_j|; every
+                                 value the chain re-evaluates is checked against
+                                 that bound, and a value outside it sets a status
+                                 bit that cg_sync_status reports as CG_ERR_BOUND */
 } cg_engine;
 
 /* Shape of a KV cache: K_l, V_l in R^{B x H x T x d} for l = 1..L
@@ -381,8 +389,10 @@ cg_status cg_spectral_stats_noalloc(const cg_kv_desc* kv, const cg_stats_desc* s
 cg_status cg_selftest_wait_timeout(int64_t limit_ns, uint32_t* result_dev, void* stream);
 
 /* Synchronizes `stream`, then reports (and clears) the device status word:
- * CG_ERR_TIMEOUT if a bounded wait ran out since the last check, CG_ERR_CUDA on
- * a pending CUDA error, else CG_OK. */
+ * CG_ERR_TIMEOUT if a bounded wait ran out since the last check, else
+ * CG_ERR_BOUND if the chain-exact tensor-core encoder met a tensor-core value
+ * outside its assumed error bound since the last check, CG_ERR_CUDA on a
+ * pending CUDA error, else CG_OK. */
 cg_status cg_sync_status(void* stream);
 
 /* Name and description of the CUDA error behind the last CG_ERR_CUDA returned

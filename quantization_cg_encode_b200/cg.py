@@ -14,7 +14,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcg.so")
 
-CG_OK, CG_ERR_INVALID, CG_ERR_UNSUPPORTED, CG_ERR_CUDA, CG_ERR_TIMEOUT, CG_ERR_TOO_LARGE = range(6)
+CG_OK, CG_ERR_INVALID, CG_ERR_UNSUPPORTED, CG_ERR_CUDA, CG_ERR_TIMEOUT, CG_ERR_TOO_LARGE, CG_ERR_BOUND = range(7)
 BLOCK_UNIFORM, KIVI = 0, 1
 ENGINE_AUTO, ENGINE_CUDA_CORES, ENGINE_CHAIN_TENSOR = 0, 1, 2
 

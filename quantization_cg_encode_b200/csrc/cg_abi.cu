@@ -346,7 +346,7 @@ cg_status cg_sync_status(void* stream) {
   if (flag) {
     e = cudaMemcpyToSymbol(cg::g_status, &zero, sizeof(zero));
     if (e != cudaSuccess) return from_cuda(e);
-    return CG_ERR_TIMEOUT;
+    return (flag & cg::kStatusTimeout) ? CG_ERR_TIMEOUT : CG_ERR_BOUND;
   }
   return CG_OK;
 }
@@ -363,6 +363,7 @@ const char* cg_status_string(cg_status s) {
     case CG_ERR_UNSUPPORTED: return "unsupported configuration";
     case CG_ERR_CUDA: return "CUDA error";
     case CG_ERR_TIMEOUT: return "device wait timed out";
+    case CG_ERR_BOUND: return "tensor-core error bound exceeded";
     case CG_ERR_TOO_LARGE: return "request exceeds the built-in scratch size";
   }
   return "unknown status";

@@ -14,6 +14,9 @@ namespace cg {
 // (defined once in cg_abi.cu; kernels receive its device address).
 // cg_sync_status() reads and clears it.
 constexpr unsigned int kStatusTimeout = 1u;
+// The chain-exact tensor-core encoder ORs kStatusBound when a value it re-evaluated with the
+// fp32 chain lay farther from its tensor-core value than the error bound its decisions assume.
+constexpr unsigned int kStatusBound = 2u;
 // Wall-time bound of any device-side wait on an asynchronous copy.
 constexpr unsigned long long kWaitNs = 2000000000ull;
 

@@ -35,7 +35,11 @@
 //     delta = (A + 2^-21 Q)/s (1 + 2^-18) from the nearest rounding boundary
 //     k + 1/2, which bounds |t_tc - t_exact|; the few values within delta are
 //     re-evaluated with the chain and quantized again.
-// So codes, steps and zero points equal the exact encoder's bit for bit.  The
+// So codes, steps and zero points equal the exact encoder's bit for bit, as long as
+// the assumed E holds; every value the chain re-evaluates is checked against A, and
+// a value outside it ORs kStatusBound into the device status word (reported by
+// cg_sync_status as CG_ERR_BOUND), so a violation on real data does not pass
+// silently.  The
 // optional fp32 gauged output holds the values actually quantized (y_tc, with
 // the chain's value wherever it was evaluated), within A of the chain.
 //
@@ -316,7 +320,7 @@ __device__ __forceinline__ float quant16(const float (&y)[16], float zf, float i
 // is reduced again.  Returns this lane's (mn, mx), exact where its block was
 // undecided.  Called by the whole warp; out of line, as it is rarely needed.
 __device__ __noinline__ float2 exact_range(const uint16_t* xrow, const float* gf, uint32_t taddr, uint32_t und,
-                                           float mn, float mx, float A) {
+                                           float mn, float mx, float A, unsigned int* status) {
   const unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31, r_own = (lane & 15) >> 1;
   uint32_t gm = 0;
@@ -346,7 +350,10 @@ __device__ __noinline__ float2 exact_range(const uint16_t* xrow, const float* gf
         const float e = chain_y(xrow, gf, r, k0);
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          if (k == k0) y[k] = e;
+          if (k == k0) {
+            if (!(fabsf(y[k] - e) <= bA)) atomicOr(status, kStatusBound);  // the assumed bound failed
+            y[k] = e;
+          }
       }
     }
     float emn, emx;
@@ -371,7 +378,8 @@ __device__ __noinline__ float2 exact_range(const uint16_t* xrow, const float* gf
 // out of line, as it is rarely needed.
 template <int BITS>
 __device__ __noinline__ void slow_group(const uint16_t* xrow, const float* gf, uint32_t taddr_r, int r, float zf,
-                                        float inv, float th, bool tile_ok, uint8_t* crow_r, float* grow) {
+                                        float inv, float th, float A, bool tile_ok, uint8_t* crow_r, float* grow,
+                                        unsigned int* status) {
   constexpr int QMAX = (1 << BITS) - 1;
   const unsigned FULL = 0xffffffffu;
   float y[16];
@@ -401,6 +409,7 @@ __device__ __noinline__ void slow_group(const uint16_t* xrow, const float* gf, u
 #pragma unroll
       for (int k = 0; k < 16; ++k)
         if (k == k0) {
+          if (!(fabsf(y[k] - e) <= A)) atomicOr(status, kStatusBound);  // the assumed bound failed
           rb[k] = rr;
           y[k] = e;
         }
@@ -758,7 +767,7 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
         }
         const uint32_t und = __ballot_sync(FULL, (lane & 1) == 0 && !decided && tile_ok);
         if (und) {
-          const float2 e = exact_range(xrow, gf, taddr, und, mn, mx, A);
+          const float2 e = exact_range(xrow, gf, taddr, und, mn, mx, A, a.status);
           mn = e.x;
           mx = e.y;
         }
@@ -802,13 +811,15 @@ __global__ void __launch_bounds__(512, 1)  // 448 threads; the bound caps regist
           const float zf = __shfl_sync(FULL, qp.zf, src);
           const float inv = __shfl_sync(FULL, qp.inv, src);
           const float th = __shfl_sync(FULL, thr, src);
+          const float Ab = __shfl_sync(FULL, A, src);
           tmem_wait_ld_into<16>(y);
           uint32_t rb[16];
           const float fmx = quant16<false, QMAX>(y, zf, inv, rb);
           float* grow = a.gauged ? a.gauged + (slice * a.k.T + tok) * D + 16 * r : nullptr;
           if (__any_sync(FULL, tile_ok && (th < -2.0f || fmx >= th))) {
             // a block needs clamping or holds values near a rounding boundary
-            slow_group<BITS>(xrow, gf, taddr + 16 * r, r, zf, inv, th, tile_ok, crow + r * (32 * BITS), grow);
+            slow_group<BITS>(xrow, gf, taddr + 16 * r, r, zf, inv, th, Ab, tile_ok, crow + r * (32 * BITS), grow,
+                             a.status);
           } else if (tile_ok) {
             store_row16<BITS>(crow + r * (32 * BITS), rb);
             if (grow) {

@@ -32,6 +32,7 @@ def test_version_and_status_strings():
     assert cg.status_string(cg.CG_OK) == "ok"
     assert "invalid" in cg.status_string(cg.CG_ERR_INVALID)
     assert "timed out" in cg.status_string(cg.CG_ERR_TIMEOUT)
+    assert "error bound" in cg.status_string(cg.CG_ERR_BOUND)
 
 
 @pytest.mark.parametrize("bits,g,w", [(3, 16, 16), (4, 16, 16), (6, 16, 16), (4, 16, 128), (4, 128, 128), (2, 8, 8)])

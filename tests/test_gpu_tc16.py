@@ -126,3 +126,37 @@ def test_non_orthogonal_gauge_is_evaluated_exactly():
     G32[0, 1] = np.random.default_rng(13).standard_normal(G32[0, 1].shape).astype(np.float32) * 0.3
     _, _, _, ref, y = _check(kv, G32, 4)
     assert np.array_equal(y, ref["y"]), "non-orthogonal gauge: every value from the chain"
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_inputs_built_against_the_error_bound(bits):
+    """Inputs built to attack the assumed accumulation bound (|y_tc - x.G_i| <= 2^-20
+    sum_j |G_ij x_j|): rows whose gauged values cancel heavily (x = bf16(G^T v) with one
+    large entry in v, so sum |G_ij x_j| is about 2^9 times most |y_i|); bf16 values whose
+    exponents span 2^-20 .. 2^20 inside one 16-vector; a near-identity gauge with tiny
+    off-diagonals; and outlier channels at 10^3 times the rest.  Codes, steps and zero
+    points must equal the oracle's chain bit for bit, and no re-evaluated value may lie
+    outside the bound (cg_sync_status, called by run_encode, would report CG_ERR_BOUND)."""
+    need_gpu()
+    L, B, H, T, d = 1, 1, 4, 256, 128
+    rng = np.random.default_rng(100 + bits)
+    G32 = _oracle_G(L, H, sigma=0.1, seed=bits)
+    G32[0, :, 2] = _oracle_G(L, H, sigma=1e-4, seed=7)[0, :, 2]        # near identity, tiny off-diagonals
+    x = np.zeros((L, 2, B, H, T, d), np.float32)
+    # head 0: heavy cancellation, y = G x close to a one-hot v per 16-vector
+    for s in range(2):
+        for r in range(8):
+            v = rng.standard_normal((T, 16)) * 1e-3
+            v[np.arange(T), rng.integers(0, 16, T)] = rng.choice([-1.0, 1.0], T) * 10.0 ** rng.uniform(0, 3, T)
+            x[0, s, 0, 0, :, 16 * r:16 * r + 16] = v @ G32[0, s, 0, r].astype(np.float64)   # x = G^T v per row
+    # head 1: exponents spread over 2^-20 .. 2^20 inside each 16-vector, random signs
+    x[0, :, 0, 1] = rng.choice([-1.0, 1.0], (2, T, d)) * 2.0 ** rng.uniform(-20, 20, (2, T, d))
+    # head 2: near-identity gauge on ordinary data; head 3: outlier channels at 10^3 x
+    x[0, :, 0, 2] = rng.standard_normal((2, T, d))
+    x[0, :, 0, 3] = rng.standard_normal((2, T, d))
+    x[0, :, 0, 3, :, [5, 40, 77, 126]] *= 1000.0
+    kv = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    _, _, _, ref, y = _check(kv, G32, bits)
+    cg.cg_sync_status()
+    err = _block_error(y, np.asarray(ref["y"], dtype=np.float64))
+    assert err <= BOUND, err
