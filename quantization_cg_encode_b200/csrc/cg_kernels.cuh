@@ -42,9 +42,11 @@ unsigned int* device_status_word();
 cg_status validate_stats(const cg_kv_desc* kv, const cg_stats_desc* st);
 bool spectral_tmem_supported(const KvGeom& k, int x_fp32);
 int spectral_tmem_pieces(const KvGeom& k);
-cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G, float lambda_f, float lambda_r,
-                                 float tau, float* lfreq, float* lrate, float* dg_part, unsigned int* status,
-                                 int num_sms, cudaStream_t st);
+// fp32 input is supported for the statistics without dL/dG (dg_part == nullptr).
+cudaError_t launch_spectral_tmem(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f,
+                                 float lambda_r, float tau, float* lfreq, float* lrate, float* dg_part,
+                                 unsigned int* status, int num_sms, cudaStream_t st);
+bool spectral_fwd_f32_supported(const KvGeom& k);
 cudaError_t launch_spectral_generic(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f,
                                     float lambda_r, float tau, float* lfreq, float* lrate, float* dg_part,
                                     int num_sms, cudaStream_t st);
@@ -83,6 +85,7 @@ cudaError_t launch_decode_attention(AttnArgs a, cudaStream_t st);
 // 2-D TMA tensor map over a row-major bf16 [rows][cols] array (box_cols x
 // box_rows boxes, 128-byte swizzle); `out` points to a CUtensorMap.
 bool make_tmap_2d_bf16(void* out, const void* base, uint64_t rows, uint64_t cols, int box_cols, int box_rows);
+bool make_tmap_2d_f32(void* out, const void* base, uint64_t rows, uint64_t cols, int box_cols, int box_rows);
 cudaError_t launch_gauge_build(const float* A, float* G, int n_mats, int g, cudaStream_t st);
 cudaError_t launch_gauge_grad(const float* A, const float* dG, float* dA, int n_mats, int g, cudaStream_t st);
 cudaError_t launch_adamw(float* p, const float* grad, float* m, float* v, long long n, float lr, float b1, float b2,

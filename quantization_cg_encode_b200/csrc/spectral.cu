@@ -566,8 +566,9 @@ cudaError_t launch_spectral(const KvGeom& k, int x_fp32, const void* x, const fl
   a.dg_part = reinterpret_cast<float*>(workspace);
   a.status = status;
   cudaError_t e;
-  if (spectral_tmem_supported(k, x_fp32)) {  // bf16 input: the gauge folded into the channel DCT
-    e = launch_spectral_tmem(k, x, G, lambda_f, lambda_r, tau, lfreq, lrate, dG ? a.dg_part : nullptr, status,
+  if (spectral_tmem_supported(k, x_fp32) || (x_fp32 && !dG && spectral_fwd_f32_supported(k))) {
+    // the gauge folded into the channel DCT (fp32 input: statistics only, x split into bf16 hi + lo)
+    e = launch_spectral_tmem(k, x_fp32, x, G, lambda_f, lambda_r, tau, lfreq, lrate, dG ? a.dg_part : nullptr, status,
                              num_sms, st);
   } else if (k.d == kD && k.T % kTile == 0) {
     e = cudaFuncSetAttribute(spectral_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSpecSmem);

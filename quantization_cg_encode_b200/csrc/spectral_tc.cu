@@ -706,29 +706,44 @@ namespace {
 constexpr uint32_t kFColM0 = 0, kFColM1 = 384, kFColU1 = 128;
 __device__ __forceinline__ uint32_t fwd_mcol(int q) { return (q & 1) ? kFColM1 : kFColM0; }
 constexpr int kRedPitch = 132;  // [12][kRedPitch] partial sums of a tile half, by channel frequency v
-constexpr int kFwdSmem = 1024 + kStages * kXBytes + 2 * 8192 + 2 * 2 * 12 * kRedPitch * 4 + kCosTab * 4 + 256;
+// bf16 input: a 4-stage ring of bf16 tiles, block sums finished in shared memory.  fp32 input:
+// a 2-stage ring of fp32 tiles (four 32-channel TMA boxes each), the current tile split by the
+// workers into bf16 hi and lo tiles (x = hi + lo to 2^-17), block sums by the warp butterfly.
+template <bool F32>
+struct FwdCfg {
+  static constexpr int NST = F32 ? 2 : kStages;
+  static constexpr int STAGE = F32 ? 4 * 16384 : kXBytes;
+  static constexpr int CONV = F32 ? 2 * kXBytes : 0;
+  static constexpr int RED = F32 ? 2 * 2 * 4 * 12 : 2 * 2 * 12 * kRedPitch;  // floats
+  static constexpr int SMEM = 1024 + NST * STAGE + CONV + 2 * 8192 + RED * 4 + kCosTab * 4 + 256;
+};
 
 
 }  // namespace
 
+template <bool F32>
 __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_constant__ CUtensorMap tmap, TmArgs a) {
+  using C = FwdCfg<F32>;
+  constexpr int NST = C::NST;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* xs = base;                                      // ring of x tiles
-  float* gs = reinterpret_cast<float*>(xs + kStages * kXBytes);  // 2 x [8][16][16] G
-  float* red = reinterpret_cast<float*>(gs + 2 * 2048);          // [2 tile parity][2 half][12][kRedPitch]
-  float* cosk = red + 2 * 2 * 12 * kRedPitch;                    // cos(k pi / 256)
+  unsigned char* xs = base;                                  // ring of input tiles
+  unsigned char* cvt = xs + NST * C::STAGE;                  // fp32 input: bf16 hi tile, then lo tile
+  float* gs = reinterpret_cast<float*>(cvt + C::CONV);       // 2 x [8][16][16] G
+  float* red = gs + 2 * 2048;                                // block sums (see FwdCfg)
+  float* cosk = red + C::RED;                                // cos(k pi / 256)
   uint64_t* bars = reinterpret_cast<uint64_t*>(cosk + kCosTab);
   uint64_t* x_full = bars;
-  uint64_t* x_empty = bars + kStages;
-  uint64_t* g_full = bars + 2 * kStages;  // [2]
+  uint64_t* x_empty = bars + NST;
+  uint64_t* g_full = bars + 2 * NST;      // [2]
   uint64_t* g_empty = g_full + 2;         // [2]
   uint64_t* m_full = g_empty + 2;         // [2]
   uint64_t* m_empty = m_full + 2;         // [2]
   uint64_t* u_full = m_empty + 2;         // [2]
   uint64_t* u_empty = u_full + 2;         // [2]
   uint64_t* mma_done = u_empty + 2;
-  uint32_t* tmem_base = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* conv_full = mma_done + 1;     // fp32 input: the current tile's hi and lo tiles are written
+  uint32_t* tmem_base = reinterpret_cast<uint32_t*>(conv_full + 1);
   volatile uint32_t* abort_flag = tmem_base + 1;
   auto wait = [&](uint64_t* bar, uint32_t parity) {
     if (*abort_flag) return;
@@ -742,10 +757,11 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
   const int n_t = (int)(total * (blockIdx.x + 1) / gridDim.x - g0);  // tiles of this CTA
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&x_full[s], 1);
-      mbar_init(&x_empty[s], 1);
+      mbar_init(&x_empty[s], F32 ? kWorkerWarps : 1);  // freed by the split (fp32) or the GEMM (bf16)
     }
+    mbar_init(conv_full, kWorkerWarps);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&g_full[s], 1);
       mbar_init(&g_empty[s], kWorkerWarps);
@@ -785,19 +801,24 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
           mbar_arrive_expect_tx(&g_full[gb], 8192);
           bulk_g2s(gs + gb * 2048, a.G + gauge_set(l, sk, h, a.k) * 2048, 8192, &g_full[gb]);
         }
-        const int s = i % kStages;
-        wait(&x_empty[s], ((uint32_t)(i / kStages) & 1u) ^ 1u);
-        mbar_arrive_expect_tx(&x_full[s], kXBytes);
+        const int s = i % NST;
+        wait(&x_empty[s], ((uint32_t)(i / NST) & 1u) ^ 1u);
+        mbar_arrive_expect_tx(&x_full[s], C::STAGE);
         const int row0 = (int)(gt * kTile);
-        tma_load_2d(xs + s * kXBytes, &tmap, 0, row0, &x_full[s]);
-        tma_load_2d(xs + s * kXBytes + 16384, &tmap, 64, row0, &x_full[s]);
+        if constexpr (F32) {  // four boxes of 32 fp32 channels (128-byte rows)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) tma_load_2d(xs + s * C::STAGE + b * 16384, &tmap, 32 * b, row0, &x_full[s]);
+        } else {
+          tma_load_2d(xs + s * C::STAGE, &tmap, 0, row0, &x_full[s]);
+          tma_load_2d(xs + s * C::STAGE + 16384, &tmap, 64, row0, &x_full[s]);
+        }
         issued = i + 1;
       }
       // Drain: the last copy into every stage and G buffer has landed before the
       // CTA can exit (immediate unless a wait above gave up).
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int last = ((issued - 1 - s) / kStages) * kStages + s;
-        mbar_wait(&x_full[s], (uint32_t)(last / kStages) & 1u, a.status);
+      for (int s = 0; s < NST && s < issued; ++s) {
+        const int last = ((issued - 1 - s) / NST) * NST + s;
+        mbar_wait(&x_full[s], (uint32_t)(last / NST) & 1u, a.status);
       }
       for (int q = ls - 1 < 0 ? 0 : ls - 1; q <= ls; ++q) mbar_wait(&g_full[q & 1], (uint32_t)(q >> 1) & 1u, a.status);
     }
@@ -806,26 +827,38 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
       int lsm = -1;
       for (int i = 0; i < n_t && !*abort_flag; ++i) {  // after a wait gave up, nothing more is issued
         const long long gt = g0 + i;
-        const int j = (int)(gt % tiles), s = i % kStages, ub = i & 1;
+        const int j = (int)(gt % tiles), s = i % NST, ub = i & 1;
         if (i == 0 || j == 0) {
           ++lsm;
           // slice lsm's M (with a gauge, buffer lsm & 1; without, one M in buffer 0)
           if (a.has_g || i == 0) wait(&m_full[lsm & 1], (uint32_t)(a.has_g ? lsm >> 1 : 0) & 1u);
         }
-        wait(&x_full[s], (uint32_t)(i / kStages) & 1u);
+        if constexpr (F32) wait(conv_full, (uint32_t)i & 1u);  // tile i's hi and lo tiles
+        else wait(&x_full[s], (uint32_t)(i / NST) & 1u);
         wait(&u_empty[ub], ((uint32_t)(i >> 1) & 1u) ^ 1u);
         fence_after();
-        const uint32_t xa = smem_u32(xs + s * kXBytes);
         const uint32_t d = tmem + kFColU1 + 128 * ub;
         const uint32_t mc = tmem + fwd_mcol(a.has_g ? lsm : 0);
+        if constexpr (F32) {  // U1^T = M_hi x_hi + M_lo x_hi + M_hi x_lo
+          const uint32_t ha = smem_u32(cvt), la = smem_u32(cvt + kXBytes);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t bd = kdesc(xa + (k >> 2) * 16384 + (k & 3) * 32);
-          mma_ts(d, mc + 8 * k, bd, idesc(false), k > 0);
-          mma_ts(d, mc + 64 + 8 * k, bd, idesc(false), 1);
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t ko = (k >> 2) * 16384 + (k & 3) * 32;
+            mma_ts(d, mc + 8 * k, kdesc(ha + ko), idesc(false), k > 0);
+            mma_ts(d, mc + 64 + 8 * k, kdesc(ha + ko), idesc(false), 1);
+            mma_ts(d, mc + 8 * k, kdesc(la + ko), idesc(false), 1);
+          }
+        } else {
+          const uint32_t xa = smem_u32(xs + s * C::STAGE);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t bd = kdesc(xa + (k >> 2) * 16384 + (k & 3) * 32);
+            mma_ts(d, mc + 8 * k, bd, idesc(false), k > 0);
+            mma_ts(d, mc + 64 + 8 * k, bd, idesc(false), 1);
+          }
         }
         commit(&u_full[ub]);
-        commit(&x_empty[s]);
+        if constexpr (!F32) commit(&x_empty[s]);
         if (a.has_g && (j == tiles - 1 || i == n_t - 1)) commit(&m_empty[lsm & 1]);
       }
       commit(mma_done);
@@ -870,7 +903,42 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
         if (a.has_g) mbar_arrive(&g_empty[q & 1]);
       }
     };
+    // fp32 input: split tile ti (its stage of the ring) into the bf16 hi and lo tiles the
+    // GEMM reads, in the same swizzled K-major layout as a bf16 TMA tile.  Worker wid takes
+    // row wid / 2, channels 64 (wid & 1) .. + 63: 16 fp32 chunks of 16 bytes (chunk c of a
+    // 32-channel box at position c ^ (row & 7)) become 8 bf16 chunks in each tile.
+    auto split_tile = [&](int ti) {
+      const int s = ti % NST;
+      wait(&x_full[s], (uint32_t)(ti / NST) & 1u);
+      const int wid = threadIdx.x - 64, r = wid >> 1, hh = wid & 1;
+      const unsigned char* src = xs + s * C::STAGE + r * 128;
+      unsigned char* hi_t = cvt + hh * 16384 + r * 128;
+      unsigned char* lo_t = hi_t + kXBytes;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {  // bf16 chunk q: channels 64 hh + 8 q .. + 7
+        const int b = 2 * hh + (q >> 2), c0 = 2 * (q & 3);  // fp32 box, first 4-channel chunk in it
+        const float4 f0 = *reinterpret_cast<const float4*>(src + b * 16384 + ((c0 ^ (r & 7)) << 4));
+        const float4 f1 = *reinterpret_cast<const float4*>(src + b * 16384 + (((c0 + 1) ^ (r & 7)) << 4));
+        uint4 h, l;
+        split2(f0.x, f0.y, h.x, l.x);
+        split2(f0.z, f0.w, h.y, l.y);
+        split2(f1.x, f1.y, h.z, l.z);
+        split2(f1.z, f1.w, h.w, l.w);
+        const int o = (q ^ (r & 7)) << 4;
+        *reinterpret_cast<uint4*>(hi_t + o) = h;
+        *reinterpret_cast<uint4*>(lo_t + o) = l;
+      }
+      fence_proxy_async_smem();  // the tiles are read by the tensor cores
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(conv_full);
+        mbar_arrive(&x_empty[s]);
+      }
+    };
     if (n_t > 0) build_m(0);
+    if constexpr (F32) {
+      if (n_t > 0) split_tile(0);
+    }
     int ls = 0;
     for (int i = 0; i < n_t; ++i) {
       const long long gt = g0 + i;
@@ -888,6 +956,11 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&u_empty[ub]);
+      // fp32 input: tile i's GEMM is done with the hi and lo tiles, so tile i + 1 is split
+      // now and its GEMM overlaps this tile's statistics
+      if constexpr (F32) {
+        if (i + 1 < n_t) split_tile(i + 1);
+      }
       float part[12];  // per block kb: E, F, R at 3 kb
 #pragma unroll
       for (int p = 0; p < 2; ++p) {  // blocks 2 p and 2 p + 1 as fp32 pairs
@@ -901,28 +974,44 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
         part[6 * p + 4] = F.y;
         part[6 * p + 5] = R.y;
       }
-      float* rb = red + ((i & 1) * 2 + hf) * (12 * kRedPitch);
-#pragma unroll
-      for (int q = 0; q < 12; ++q) rb[q * kRedPitch + v] = part[q];
-      named_bar_sync(2 + hf, 128);
-      // One warp per half (channel quarter 3 or 2: not the SMSPs of the producer and MMA
-      // warps) finishes the sums: lane 8 kb + s adds v = 16 s .. 16 s + 15 of block kb.
-      if (wq == (hf ? 2 : 3)) {
-        const int kb = lane >> 3, sx = lane & 7;
-        float acc[3];
-#pragma unroll
-        for (int c = 0; c < 3; ++c) {
-          const float4* src = reinterpret_cast<const float4*>(rb + (3 * kb + c) * kRedPitch + 16 * sx);
-          const float4 a0 = src[0], a1 = src[1], a2 = src[2], a3 = src[3];
-          acc[c] = (((a0.x + a0.y) + (a0.z + a0.w)) + ((a1.x + a1.y) + (a1.z + a1.w))) +
-                   (((a2.x + a2.y) + (a2.z + a2.w)) + ((a3.x + a3.y) + (a3.z + a3.w)));
-#pragma unroll
-          for (int o = 1; o < 8; o <<= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
-        }
-        if (sx == 0) {
+      if constexpr (F32) {  // the halving butterfly, then the quarters' sums
+        const float tot = warp_sum12(part, lane);
+        float* rb = red + ((i & 1) * 2 + hf) * 48;
+        if (!(lane & 1) && (lane >> 1) < 12) rb[wq * 12 + (lane >> 1)] = tot;
+        named_bar_sync(2 + hf, 128);
+        if (wq == 0 && lane < 4) {
+          const int kb = lane;
+          const float E = (rb[0 * 12 + 3 * kb] + rb[1 * 12 + 3 * kb]) + (rb[2 * 12 + 3 * kb] + rb[3 * 12 + 3 * kb]);
+          const float F = (rb[0 * 12 + 3 * kb + 1] + rb[1 * 12 + 3 * kb + 1]) + (rb[2 * 12 + 3 * kb + 1] + rb[3 * 12 + 3 * kb + 1]);
+          const float R = (rb[0 * 12 + 3 * kb + 2] + rb[1 * 12 + 3 * kb + 2]) + (rb[2 * 12 + 3 * kb + 2] + rb[3 * 12 + 3 * kb + 2]);
           const long long blk = gt * 8 + 4 * hf + kb;
-          a.lfreq[blk] = acc[0] > 0.0f ? acc[1] / acc[0] : 0.0f;
-          a.lrate[blk] = acc[2] * 0.69314718055994531f / (16.0f * kD);
+          a.lfreq[blk] = E > 0.0f ? F / E : 0.0f;
+          a.lrate[blk] = R * 0.69314718055994531f / (16.0f * kD);
+        }
+      } else {
+        float* rb = red + ((i & 1) * 2 + hf) * (12 * kRedPitch);
+#pragma unroll
+        for (int q = 0; q < 12; ++q) rb[q * kRedPitch + v] = part[q];
+        named_bar_sync(2 + hf, 128);
+        // One warp per half (channel quarter 3 or 2: not the SMSPs of the producer and MMA
+        // warps) finishes the sums: lane 8 kb + s adds v = 16 s .. 16 s + 15 of block kb.
+        if (wq == (hf ? 2 : 3)) {
+          const int kb = lane >> 3, sx = lane & 7;
+          float acc[3];
+#pragma unroll
+          for (int c = 0; c < 3; ++c) {
+            const float4* src = reinterpret_cast<const float4*>(rb + (3 * kb + c) * kRedPitch + 16 * sx);
+            const float4 a0 = src[0], a1 = src[1], a2 = src[2], a3 = src[3];
+            acc[c] = (((a0.x + a0.y) + (a0.z + a0.w)) + ((a1.x + a1.y) + (a1.z + a1.w))) +
+                     (((a2.x + a2.y) + (a2.z + a2.w)) + ((a3.x + a3.y) + (a3.z + a3.w)));
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
+          }
+          if (sx == 0) {
+            const long long blk = gt * 8 + 4 * hf + kb;
+            a.lfreq[blk] = acc[0] > 0.0f ? acc[1] / acc[0] : 0.0f;
+            a.lrate[blk] = acc[2] * 0.69314718055994531f / (16.0f * kD);
+          }
         }
       }
     }
@@ -936,13 +1025,17 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
 }
 
 bool spectral_tmem_supported(const KvGeom& k, int x_fp32) { return !x_fp32 && k.d == kD && k.T % kTile == 0; }
+bool spectral_fwd_f32_supported(const KvGeom& k) { return k.d == kD && k.T % kTile == 0; }
 int spectral_tmem_pieces(const KvGeom& k) { return (k.d == kD && k.T % (2 * kTile) == 0) ? 2 : 1; }
 
-cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G, float lambda_f, float lambda_r,
-                                 float tau, float* lfreq, float* lrate, float* dg_part, unsigned int* status,
-                                 int num_sms, cudaStream_t st) {
+cudaError_t launch_spectral_tmem(const KvGeom& k, int x_fp32, const void* x, const float* G, float lambda_f,
+                                 float lambda_r, float tau, float* lfreq, float* lrate, float* dg_part,
+                                 unsigned int* status, int num_sms, cudaStream_t st) {
+  if (x_fp32 && dg_part) return cudaErrorInvalidValue;  // fp32 input: statistics only
   alignas(64) CUtensorMap tmap;
-  if (!make_tmap_2d_bf16(&tmap, x, (uint64_t)k.slices() * k.T, kD, 64, kTile)) return cudaErrorInvalidValue;
+  const uint64_t rows = (uint64_t)k.slices() * k.T;
+  if (x_fp32 ? !make_tmap_2d_f32(&tmap, x, rows, kD, 32, kTile) : !make_tmap_2d_bf16(&tmap, x, rows, kD, 64, kTile))
+    return cudaErrorInvalidValue;
   TmArgs a;
   a.k = k;
   a.has_g = G != nullptr;
@@ -959,11 +1052,13 @@ cudaError_t launch_spectral_tmem(const KvGeom& k, const void* x, const float* G,
   a.dg_part = dg_part;
   a.status = status;
   if (dg_part == nullptr) {  // statistics only: tile-balanced ranges
-    cudaError_t e = cudaFuncSetAttribute(spectral_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmem);
+    auto kern = x_fp32 ? spectral_fwd_kernel<true> : spectral_fwd_kernel<false>;
+    const int smem = x_fp32 ? FwdCfg<true>::SMEM : FwdCfg<false>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const long long tiles = k.slices() * (k.T / kTile);
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-    spectral_fwd_kernel<<<grid, kThreads, kFwdSmem, st>>>(tmap, a);
+    kern<<<grid, kThreads, smem, st>>>(tmap, a);
     return cudaGetLastError();
   }
   a.pieces = spectral_tmem_pieces(k);

@@ -190,6 +190,29 @@ def test_stats_forward_tile_ranges(gauged):
     _check(ref, lf, lr, tot)
 
 
+@pytest.mark.parametrize("gauged", [True, False])
+def test_stats_fp32_input_tile_ranges(gauged):
+    """fp32 input (already gauged, or with a g = 16 gauge applied in the kernel) takes the
+    tensor-core statistics kernel too: each tile is split into bf16 hi + lo in shared
+    memory and the channel GEMM runs three terms.  512 tiles of 4 x 2 x 1 x 4 slices of
+    2048 tokens over at most 148 CTAs: ranges cross slices and wrap the 2-stage fp32 ring.
+    Values span a wide range (N(0, 3) with 100x outlier channels and a 1e-3 scaled head),
+    every block against the oracle."""
+    need_gpu()
+    L, B, H, T, d = 4, 1, 4, 2048, 128
+    g = torch.Generator().manual_seed(21)
+    x = torch.randn((L, 2, B, H, T, d), generator=g) * 3
+    x[..., [7, 90]] *= 100.0
+    x[:, :, :, 3] *= 1e-3
+    x[0, 0, 0, 1, 16:32] = 0.0          # an all-zero block
+    x = x.cuda().contiguous()
+    G = oracle_gauge(synth.gauge_params(L, H, 8, 16, sigma=0.1, seed=21)) if gauged else None
+    lf, lr, tot, _ = run_stats(x, G, False, True)
+    Gn = G.cpu().numpy().astype(np.float64) if gauged else None
+    ref = sp.spectral_stats(x.cpu().numpy().astype(np.float64), Gn)
+    _check(ref, lf, lr, tot)
+
+
 @pytest.mark.parametrize("want_grad", [False, True])
 def test_stats_tiny_config_d64(want_grad):
     """The small reference cache (1 x 2 x 1 x 2 x 1024 x 64, g = 16): the statistic spans
