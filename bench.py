@@ -346,6 +346,11 @@ def measure_rows(args, cg, synth, torch, kv, G16, stream, dev, rank):
         ws = torch.empty(max(cg.cg_spectral_workspace_size(kvd, st, True), 16), dtype=torch.uint8, device=dev)
         rec("stats_fwd", _time(lambda: cg.cg_spectral_stats(kvd, st, kv, G16, lf, lr, tot, None, ws, stream=stream), stream), 2.0, 2 * 144 + 32)
         rec("stats_fwd_bwd", _time(lambda: cg.cg_spectral_stats(kvd, st, kv, G16, lf, lr, tot, dG, ws, stream=stream), stream), 4.0, 2 * 288 + 96)
+        # the same window as fp32 already-gauged tensors (G NULL): 4 B per value in
+        x32 = kv.float()
+        st32 = cg.StatsDesc(16, 0, 1, 1.0, 0.02, 0.04)
+        rec("stats_fwd_fp32_gauged", _time(lambda: cg.cg_spectral_stats(kvd, st32, x32, None, lf, lr, tot, None, ws, stream=stream), stream), 4.0, 2 * 144 + 32)
+        del x32
         # decode-step attention from the 4-bit cache: every layer, 32 query heads, all 4096 tokens
         codec = cg.codec_desc(g=16, bits=4)
         c, sc, z = cg.alloc_encoded(kvd, codec, device=dev)
