@@ -1,5 +1,6 @@
 // C ABI of libcg (declared in include/cg.h): argument validation, buffer
 // sizes, kernel dispatch and the device status word.
+#include <atomic>
 #include <cstring>
 
 #include "cg_kernels.cuh"
@@ -71,16 +72,21 @@ thread_local cudaError_t t_last_cuda = cudaSuccess;
 
 // Device address of the status word on the current device (looked up once
 // per device; a host-side symbol is not a device address).
+// The status word's device address on the current device, looked up once per device.
+// Concurrent first calls from several host threads may each look it up; they store the
+// same value, and the atomics make that well defined.
 unsigned int* status_word() {
-  static unsigned int* addr[64] = {nullptr};
+  static std::atomic<unsigned int*> addr[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
+  unsigned int* a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, cg::g_status) != cudaSuccess) return nullptr;
-    addr[dev] = (unsigned int*)p;
+    a = (unsigned int*)p;
+    addr[dev].store(a, std::memory_order_release);
   }
-  return addr[dev];
+  return a;
 }
 
 }  // namespace
