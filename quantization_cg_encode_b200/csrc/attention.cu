@@ -52,6 +52,18 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// 4-bit codes to exact fp16 pairs without moving single nibbles: the nibbles at bits
+// 0 and 16 of w give 1024 + n (one LOP3, then minus 1024), those at bits 4 and 20 give
+// 1024 + 16 n (then / 16 - 64, exact in fp16).
+__device__ __forceinline__ uint32_t nib_lo_pair(uint32_t w) {
+  return f16_sub1024((w & 0x000F000Fu) | 0x64006400u);
+}
+__device__ __forceinline__ uint32_t nib_hi_pair(uint32_t w) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"((w & 0x00F000F0u) | 0x64006400u), "r"(0x2C002C00u), "r"(0xD400D400u));
+  return r;
+}
+
 }  // namespace
 
 // partial[l][b][hq][split] = {m, l, o[D]} in gauge coordinates, over the token
@@ -161,15 +173,32 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
   }
   __syncthreads();
   // the B fragments of q'' (column n = g of tile tt holds q'' = q' 2^e of (term,
-  // head); k slots 2c, 2c+1 / 2c+8, 2c+9 are channels 4c, 4c+1 / 4c+2, 4c+3 of the group)
+  // head); k slots 2c, 2c+1 / 2c+8, 2c+9 are channels 4c, 4c+1 / 4c+2, 4c+3 of the group,
+  // or, for 4-bit codes, channels b, b+4 / b+1, b+5 with b = 8 (c >> 1) + 2 (c & 1): the
+  // nibble pairs a key word yields directly)
   for (int e = tid; e < NG * NT * 32; e += kAttnThreads) {
     const int ln = e & 31, tt = (e >> 5) % NT, r = (e >> 5) / NT;
     const int gg = ln >> 2, cc = ln & 3;
     const int j = NT == 2 ? gg : (gg & 3), lo = NT == 2 ? tt : (gg >> 2);
     const bool on = j < GQ;
     const float sj = on ? 1.0f / qinv[j] : 0.0f;
-    const float4 q4 = on ? *reinterpret_cast<const float4*>(qp + j * D + 16 * r + 4 * cc) : make_float4(0, 0, 0, 0);
-    const float v[4] = {q4.x * sj, q4.y * sj, q4.z * sj, q4.w * sj};
+    float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (on) {
+      const float* qg = qp + j * D + 16 * r;
+      if constexpr (BITS == 4) {
+        const int bb = 8 * (cc >> 1) + 2 * (cc & 1);
+        v[0] = qg[bb] * sj;
+        v[1] = qg[bb + 4] * sj;
+        v[2] = qg[bb + 1] * sj;
+        v[3] = qg[bb + 5] * sj;
+      } else {
+        const float4 q4 = *reinterpret_cast<const float4*>(qg + 4 * cc);
+        v[0] = q4.x * sj;
+        v[1] = q4.y * sj;
+        v[2] = q4.z * sj;
+        v[3] = q4.w * sj;
+      }
+    }
     __half hv[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -226,9 +255,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
         for (int r = 0; r < NG; ++r) {
           const uint8_t* blk = kc + (kb * NG + r) * BLK;
           uint32_t cv[2];  // rows g, g+8: codes 4c .. 4c+3 (4 BITS bits, low aligned)
-          if constexpr (BITS == 4) {
-            cv[0] = *reinterpret_cast<const uint16_t*>(blk + (bit_g >> 3));
-            cv[1] = *reinterpret_cast<const uint16_t*>(blk + (bit_g8 >> 3));
+          if constexpr (BITS == 4) {  // rows g, g+8: 8 bytes each; word c >> 1, from byte c & 1
+            cv[0] = *reinterpret_cast<const uint32_t*>(blk + 8 * g + 4 * (c >> 1)) >> (8 * (c & 1));
+            cv[1] = *reinterpret_cast<const uint32_t*>(blk + 8 * (g + 8) + 4 * (c >> 1)) >> (8 * (c & 1));
           } else if constexpr (BITS == 8) {
             cv[0] = *reinterpret_cast<const uint32_t*>(blk + (bit_g >> 3));
             cv[1] = *reinterpret_cast<const uint32_t*>(blk + (bit_g8 >> 3));
@@ -242,12 +271,21 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
             cv[1] = __funnelshift_r(w1[0], w1[1], bit_g8 & 31);
           }
           uint32_t afr[4];
-  #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            constexpr uint32_t M = (1u << BITS) - 1u;
-            const uint32_t v = cv[hh];
-            afr[hh] = f16_sub1024(0x64006400u | (v & M) | (((v >> BITS) & M) << 16));
-            afr[2 + hh] = f16_sub1024(0x64006400u | ((v >> (2 * BITS)) & M) | (((v >> (3 * BITS)) & M) << 16));
+          if constexpr (BITS == 4) {  // rows g, g+8: the word of channels 8 (c >> 1) .., from nibble 2 (c & 1)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t u = cv[hh];
+              afr[hh] = nib_lo_pair(u);      // channels b, b + 4
+              afr[2 + hh] = nib_hi_pair(u);  // channels b + 1, b + 5
+            }
+          } else {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              constexpr uint32_t M = (1u << BITS) - 1u;
+              const uint32_t v = cv[hh];
+              afr[hh] = f16_sub1024(0x64006400u | (v & M) | (((v >> BITS) & M) << 16));
+              afr[2 + hh] = f16_sub1024(0x64006400u | ((v >> (2 * BITS)) & M) | (((v >> (3 * BITS)) & M) << 16));
+            }
           }
           const float sk = __half2float(ks[kb * NG + r]);
   #pragma unroll
@@ -334,6 +372,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
     {
       constexpr int WPG = 8 / NG;  // warps per group: 1 (d = 128) or 2 (d = 64)
       const int r = warp % NG, part = warp / NG;
+      // byte g & 3 of the first word to byte 0, of the second to byte 2 (4-bit values)
+      const uint32_t vsel = (uint32_t)(g & 3) * 0x0011u + (uint32_t)(4 + (g & 3)) * 0x1100u;
       const int per = NBLK / WPG;
       float o[NT][4];
   #pragma unroll
@@ -343,30 +383,41 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
       float oz[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // zero-point terms of this thread's (channel, head) pairs
       for (int kb = part * per; kb < min(nblk, part * per + per); ++kb) {
         const uint8_t* blk = vc + (kb * NG + r) * BLK;
-        uint32_t lo2[4], hi2[4];  // per token 4c + u: codes of channels 2g, 2g+1
-  #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int bit = ((4 * c + u) * 16 + 2 * g) * BITS;
-          uint32_t v;
-          if constexpr (BITS == 4) {
-            v = blk[bit >> 3];
-          } else if constexpr (BITS == 8) {
-            v = *reinterpret_cast<const uint16_t*>(blk + (bit >> 3));
-          } else if constexpr (BITS == 2) {
-            v = (uint32_t)blk[bit >> 3] >> (bit & 7);
-          } else {
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(blk) + (bit >> 5);
-            v = __funnelshift_r(w[0], w[1], bit & 31);
-          }
-          constexpr uint32_t M = (1u << BITS) - 1u;
-          lo2[u] = v & M;
-          hi2[u] = (v >> BITS) & M;
-        }
         uint32_t afr[4];
-        afr[0] = f16_sub1024(0x64006400u | lo2[0] | (lo2[1] << 16));
-        afr[1] = f16_sub1024(0x64006400u | hi2[0] | (hi2[1] << 16));
-        afr[2] = f16_sub1024(0x64006400u | lo2[2] | (lo2[3] << 16));
-        afr[3] = f16_sub1024(0x64006400u | hi2[2] | (hi2[3] << 16));
+        if constexpr (BITS == 4) {
+          // token 4c + u is 8 bytes (16 channels); byte g holds channels 2g (low nibble) and
+          // 2g + 1: pick it from two tokens' words at once, then both nibble pairs
+          uint32_t w[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) w[u] = *reinterpret_cast<const uint32_t*>(blk + (4 * c + u) * 8 + 4 * (g >> 2));
+          const uint32_t x01 = __byte_perm(w[0], w[1], vsel), x23 = __byte_perm(w[2], w[3], vsel);
+          afr[0] = nib_lo_pair(x01);
+          afr[1] = nib_hi_pair(x01);
+          afr[2] = nib_lo_pair(x23);
+          afr[3] = nib_hi_pair(x23);
+        } else {
+          uint32_t lo2[4], hi2[4];  // per token 4c + u: codes of channels 2g, 2g+1
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int bit = ((4 * c + u) * 16 + 2 * g) * BITS;
+            uint32_t v;
+            if constexpr (BITS == 8) {
+              v = *reinterpret_cast<const uint16_t*>(blk + (bit >> 3));
+            } else if constexpr (BITS == 2) {
+              v = (uint32_t)blk[bit >> 3] >> (bit & 7);
+            } else {
+              const uint32_t* wp = reinterpret_cast<const uint32_t*>(blk) + (bit >> 5);
+              v = __funnelshift_r(wp[0], wp[1], bit & 31);
+            }
+            constexpr uint32_t M = (1u << BITS) - 1u;
+            lo2[u] = v & M;
+            hi2[u] = (v >> BITS) & M;
+          }
+          afr[0] = f16_sub1024(0x64006400u | lo2[0] | (lo2[1] << 16));
+          afr[1] = f16_sub1024(0x64006400u | hi2[0] | (hi2[1] << 16));
+          afr[2] = f16_sub1024(0x64006400u | lo2[2] | (lo2[3] << 16));
+          afr[3] = f16_sub1024(0x64006400u | hi2[2] | (hi2[3] << 16));
+        }
         const float sv = __half2float(vs[kb * NG + r]) * (1.0f / kPScale), zv = __half2float(vz[kb * NG + r]);
   #pragma unroll
         for (int tt = 0; tt < NT; ++tt) {
