@@ -271,7 +271,9 @@ cg_status cg_roundtrip_workspace_size(const cg_kv_desc* kv, uint64_t* bytes);
  *   workspace_dev / workspace_bytes: at least cg_roundtrip_workspace_size().
  * The call is ordered after earlier work on `stream`, and later work on
  * `stream` is ordered after all of it; the host buffers must stay valid and
- * unchanged until then.  Argument errors as in cg_encode; CG_ERR_UNSUPPORTED
+ * unchanged until then.  Concurrent calls on one device share the internal
+ * streams (they stay correct, each with its own workspace, but queue behind
+ * one another).  Argument errors as in cg_encode; CG_ERR_UNSUPPORTED
  * when one layer's codes, steps or zero points are not a multiple of 16 bytes
  * (the per-layer pointers must stay aligned). */
 cg_status cg_roundtrip_host(const cg_kv_desc* kv, const cg_codec_desc* codec, const void* kv_host,
