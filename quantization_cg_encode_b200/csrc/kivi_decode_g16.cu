@@ -81,6 +81,16 @@ __device__ __forceinline__ uint32_t bits_at(const unsigned char* p, int bit) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(p) + (bit >> 5);
   return __funnelshift_r(w[0], w[1], bit & 31);
 }
+// The same for a field of four codes at the offsets this decoder reads: with 2, 4 or 8
+// bits per code such a field never crosses a 32-bit word, so one word suffices.
+template <int BITS>
+__device__ __forceinline__ uint32_t field4_at(const unsigned char* p, int bit) {
+  if constexpr (BITS == 2 || BITS == 4 || BITS == 8) {
+    return reinterpret_cast<const uint32_t*>(p)[bit >> 5] >> (bit & 31);
+  } else {
+    return bits_at(p, bit);
+  }
+}
 
 }  // namespace
 
@@ -237,7 +247,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) kivi_decode_g16_kernel(CodecAr
           for (int half = 0; half < 2; ++half) {
             const int t = 4 * g4 + 2 * tt + half;  // MMA row g4 + 8 half of tile tt
             const int bit = ((t * 4 + (r >> 1)) * 32 + 16 * (r & 1) + 4 * q4) * BITS;
-            const uint32_t v = bits_at(cbuf, bit);
+            const uint32_t v = field4_at<BITS>(cbuf, bit);
             const uint32_t c0 = v & M, c1 = (v >> BITS) & M, c2 = (v >> (2 * BITS)) & M, c3 = (v >> (3 * BITS)) & M;
             // k slots 2q, 2q+1 <- channels 4q, 4q+1;  k slots 2q+8, 2q+9 <- channels 4q+2, 4q+3
             afr[half] = f16pair(c0, c1);
@@ -259,7 +269,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) kivi_decode_g16_kernel(CodecAr
           // 4 g4 .. 4 g4 + 3 of channel 16 r + 4 q4 + m are 4 BITS consecutive bits
           uint32_t w[4];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) w[m] = bits_at(cbuf, (16 * r + 4 * q4 + m) * 32 * BITS + 4 * g4 * BITS);
+          for (int m = 0; m < 4; ++m) w[m] = field4_at<BITS>(cbuf, (16 * r + 4 * q4 + m) * 32 * BITS + 4 * g4 * BITS);
           uint32_t afr[4];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
