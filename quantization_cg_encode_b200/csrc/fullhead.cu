@@ -426,6 +426,13 @@ __device__ inline FdSmem fd_carve(unsigned char* raw) {
 }
 constexpr int kFdSmem = 1024 + 4 * kBlockBytes + 256 * 4 + kDecEpi * kStgWarp + 12 * 8 + 16;
 
+// bf16 pair of the 4-bit codes at bits 0 and 16 of v: 128 + q is exact in bf16
+// (0x4300 | q), and subtracting 128 leaves q.
+__device__ __forceinline__ uint32_t bf16_nib_pair(uint32_t v) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"((v & 0x000F000Fu) | 0x43004300u), "r"(0x43004300u));
+  return r;
+}
 // bf16 bits of two codes (< 256, exact), packed low / high
 __device__ __forceinline__ uint32_t code_pair_bf16(uint32_t q0, uint32_t q1) {
   const f2_t v = f2_add(f2_make(__uint_as_float(0x4B000000u | q0), __uint_as_float(0x4B000000u | q1)),
@@ -486,7 +493,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
         slice_coords(slice, a.k, l, sk, b, h);
         const float* Gp = a.G + gauge_set(l, sk, h, a.k) * D * D;  // G[k][n]
         unsigned char* gdst = sm.gs + gb * kBlockBytes;
-        // lane owns output columns n = lane, lane+32, ...: row n of B = column n of G
+        // lane owns output columns n = lane, lane+32, ...: row n of B = column n of G.  With
+        // 4-bit codes the k slots of every 8-channel chunk hold channels 0, 4, 1, 5, 2, 6, 3, 7
+        // (the order in which the code expansion produces them); the column sums run in
+        // channel order either way.
         for (int n = lane; n < D; n += 32) {
           float cs = 0.0f;
           for (int k0 = 0; k0 < D; k0 += 8) {
@@ -497,7 +507,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
               w[e] = pack_bf16x2(g0, g1);
               cs += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xffff0000u);
             }
-            *reinterpret_cast<uint4*>(gdst + sw128_offset(n, k0)) = make_uint4(w[0], w[1], w[2], w[3]);
+            if constexpr (BITS == 4) {  // pairs (0, 4), (1, 5), (2, 6), (3, 7) of the chunk
+              const uint32_t p0 = __byte_perm(w[0], w[2], 0x5410), p1 = __byte_perm(w[0], w[2], 0x7632);
+              const uint32_t p2 = __byte_perm(w[1], w[3], 0x5410), p3 = __byte_perm(w[1], w[3], 0x7632);
+              *reinterpret_cast<uint4*>(gdst + sw128_offset(n, k0)) = make_uint4(p0, p1, p2, p3);
+            } else {
+              *reinterpret_cast<uint4*>(gdst + sw128_offset(n, k0)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
           sm.colsum[gb * 128 + n] = cs;
         }
@@ -597,14 +613,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) fullhead_decode_kernel(CodecAr
           unsigned char* adst = sm.as + ab * kBlockBytes;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {  // 16-byte chunk c = channels 8c .. 8c+7
-            uint32_t q[8];
+            uint4 w;
+            if constexpr (BITS == 4) {
+              // word c holds the chunk's 8 codes; the nibbles at bits 0 and 16 of w >> 4 e are
+              // channels e and e + 4: 128 + q as bf16 by one mask, minus 128 exactly
+              const uint32_t v = words[c];
+              w = make_uint4(bf16_nib_pair(v), bf16_nib_pair(v >> 4), bf16_nib_pair(v >> 8), bf16_nib_pair(v >> 12));
+            } else {
+              uint32_t q[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int bit = (8 * c + e) * BITS;
-              q[e] = __funnelshift_r(words[bit >> 5], words[(bit >> 5) + 1], bit & 31) & M;
+              for (int e = 0; e < 8; ++e) {
+                const int bit = (8 * c + e) * BITS;
+                q[e] = __funnelshift_r(words[bit >> 5], words[(bit >> 5) + 1], bit & 31) & M;
+              }
+              w = make_uint4(code_pair_bf16(q[0], q[1]), code_pair_bf16(q[2], q[3]), code_pair_bf16(q[4], q[5]),
+                             code_pair_bf16(q[6], q[7]));
             }
-            const uint4 w = make_uint4(code_pair_bf16(q[0], q[1]), code_pair_bf16(q[2], q[3]),
-                                       code_pair_bf16(q[4], q[5]), code_pair_bf16(q[6], q[7]));
             *reinterpret_cast<uint4*>(adst + sw128_offset(row, 8 * c)) = w;
           }
           fence_proxy_async_smem();
