@@ -188,11 +188,16 @@ __device__ __forceinline__ void idct16_pair(const float2 (&dU)[16], float2 (&s)[
 }
 
 // Per-block sums over the 16 frequencies of a thread's channel frequency v, for the
-// two blocks of a pair: E = sum U^2, F = sum r_uv U^2, R = sum log2(1 + |U| / tau)
-// (the logarithms taken two at a time, log2 p + log2 q = log2 (p q)).
+// two blocks of a pair: E = sum U^2, F = sum r_uv U^2, R = sum log2(1 + |U| / tau).
+// The logarithms are taken four at a time (log2 of the product of four arguments);
+// a product overflows only when some |U| / tau is beyond about 2^32, and then the
+// block's R is taken again two arguments at a time.
 __device__ __forceinline__ void pair_sums(const float2 (&U)[16], const float2 (&rad2)[16], float inv_tau, float2& E,
                                           float2& F, float2& R) {
-  float2 pr = make_float2(1.0f, 1.0f);
+  auto arg = [&](int u) {
+    return make_float2(__fmaf_rn(fabsf(U[u].x), inv_tau, 1.0f), __fmaf_rn(fabsf(U[u].y), inv_tau, 1.0f));
+  };
+  float2 p01 = make_float2(1.0f, 1.0f);
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
     const float2 e2 = __fmul2_rn(U[u], U[u]);
@@ -203,13 +208,19 @@ __device__ __forceinline__ void pair_sums(const float2 (&U)[16], const float2 (&
       E = __fadd2_rn(E, e2);
       F = __ffma2_rn(rad2[u], e2, F);
     }
-    const float2 g = make_float2(__fmaf_rn(fabsf(U[u].x), inv_tau, 1.0f), __fmaf_rn(fabsf(U[u].y), inv_tau, 1.0f));
-    if (u & 1) {
-      const float2 q = __fmul2_rn(pr, g);
+    if ((u & 3) == 1) p01 = __fmul2_rn(arg(u - 1), arg(u));
+    if ((u & 3) == 3) {
+      const float2 q = __fmul2_rn(p01, __fmul2_rn(arg(u - 1), arg(u)));
       const float2 l = make_float2(lg2_ftz(q.x), lg2_ftz(q.y));
-      R = u == 1 ? l : __fadd2_rn(R, l);
-    } else {
-      pr = g;
+      R = u == 3 ? l : __fadd2_rn(R, l);
+    }
+  }
+  if (!(fmaxf(R.x, R.y) < INFINITY)) {
+#pragma unroll
+    for (int u = 0; u < 16; u += 2) {
+      const float2 q = __fmul2_rn(arg(u), arg(u + 1));
+      const float2 l = make_float2(lg2_ftz(q.x), lg2_ftz(q.y));
+      R = u == 0 ? l : __fadd2_rn(R, l);
     }
   }
 }
@@ -711,10 +722,15 @@ constexpr int kRedPitch = 132;  // [12][kRedPitch] partial sums of a tile half, 
 // workers into bf16 hi and lo tiles (x = hi + lo to 2^-17), block sums by the warp butterfly.
 template <bool F32>
 struct FwdCfg {
+  static constexpr int WW = F32 ? 8 : 16;         // worker warps: 4 lane quarters x PARTS token parts
+  static constexpr int PARTS = WW / 4;
+  static constexpr int TPP = kTile / PARTS;       // tokens of a tile per part (64 or 32)
+  static constexpr int BPP = TPP / 16;            // 16-token blocks per part
+  static constexpr int THREADS = (2 + WW) * 32;
   static constexpr int NST = F32 ? 2 : kStages;
   static constexpr int STAGE = F32 ? 4 * 16384 : kXBytes;
   static constexpr int CONV = F32 ? 2 * kXBytes : 0;
-  static constexpr int RED = F32 ? 2 * 2 * 4 * 12 : 2 * 2 * 12 * kRedPitch;  // floats
+  static constexpr int RED = F32 ? 2 * 2 * 4 * 12 : 2 * PARTS * 3 * BPP * kRedPitch;  // floats
   static constexpr int SMEM = 1024 + NST * STAGE + CONV + 2 * 8192 + RED * 4 + kCosTab * 4 + 256;
 };
 
@@ -722,9 +738,9 @@ struct FwdCfg {
 }  // namespace
 
 template <bool F32>
-__global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_constant__ CUtensorMap tmap, TmArgs a) {
+__global__ void __launch_bounds__(FwdCfg<F32>::THREADS, 1) spectral_fwd_kernel(const __grid_constant__ CUtensorMap tmap, TmArgs a) {
   using C = FwdCfg<F32>;
-  constexpr int NST = C::NST;
+  constexpr int NST = C::NST, WW = C::WW, PARTS = C::PARTS, TPP = C::TPP, BPP = C::BPP;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char* xs = base;                                  // ring of input tiles
@@ -759,24 +775,24 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&x_full[s], 1);
-      mbar_init(&x_empty[s], F32 ? kWorkerWarps : 1);  // freed by the split (fp32) or the GEMM (bf16)
+      mbar_init(&x_empty[s], F32 ? WW : 1);  // freed by the split (fp32) or the GEMM (bf16)
     }
-    mbar_init(conv_full, kWorkerWarps);
+    mbar_init(conv_full, WW);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&g_full[s], 1);
-      mbar_init(&g_empty[s], kWorkerWarps);
+      mbar_init(&g_empty[s], WW);
       mbar_init(&u_full[s], 1);
-      mbar_init(&u_empty[s], kWorkerWarps);
+      mbar_init(&u_empty[s], WW);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&m_full[s], kWorkerWarps);
+      mbar_init(&m_full[s], WW);
       mbar_init(&m_empty[s], 1);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
-  if (warp >= 2) fill_cos_table(cosk, threadIdx.x - 64);
+  if (warp >= 2 && threadIdx.x < 64 + 256) fill_cos_table(cosk, threadIdx.x - 64);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base)), "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -789,9 +805,10 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
   if (warp == 0) {
     if (lane == 0) {
       int ls = -1, issued = 0;
+      int j = (int)(g0 % tiles) - 1;  // tile index within its slice, advanced per tile
       for (int i = 0; i < n_t && !*abort_flag; ++i) {  // after a wait gave up, nothing more is issued
         const long long gt = g0 + i;
-        const int j = (int)(gt % tiles);
+        if (++j == tiles) j = 0;
         if (a.has_g && (i == 0 || j == 0)) {
           ++ls;
           const int gb = ls & 1;
@@ -825,9 +842,10 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
   } else if (warp == 1) {
     if (lane == 0) {
       int lsm = -1;
+      int j = (int)(g0 % tiles) - 1;
       for (int i = 0; i < n_t && !*abort_flag; ++i) {  // after a wait gave up, nothing more is issued
-        const long long gt = g0 + i;
-        const int j = (int)(gt % tiles), s = i % NST, ub = i & 1;
+        if (++j == tiles) j = 0;
+        const int s = i % NST, ub = i & 1;
         if (i == 0 || j == 0) {
           ++lsm;
           // slice lsm's M (with a gauge, buffer lsm & 1; without, one M in buffer 0)
@@ -865,6 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
       mbar_wait(mma_done, 0u, a.status);
     }
   } else {
+    // worker warp: lane quarter wq (tensor-memory lanes 32 wq ..), token part hf of the tile
     const int wq = warp & 3, hf = (warp - 2) >> 2;
     const int v = 32 * wq + lane;
     const uint32_t lrow = (uint32_t)(32 * wq) << 16;
@@ -888,8 +907,8 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
       const float* G = gs + (q & 1) * 2048;
       const uint32_t mc = tmem + lrow + fwd_mcol(q);
 #pragma unroll 1
-      for (int r4 = 0; r4 < 4; ++r4) {
-        const int r = 4 * hf + r4;
+      for (int r4 = 0; r4 < 8 / PARTS; ++r4) {  // channel groups 16 r .. 16 r + 15 of this part
+        const int r = (8 / PARTS) * hf + r4;
         uint32_t h8[8], l8[8];
         m_group(cosk, G, a.has_g, v, r, h8, l8);
         st8(mc + 8 * r, h8);
@@ -940,18 +959,20 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
       if (n_t > 0) split_tile(0);
     }
     int ls = 0;
+    int j = (int)(g0 % tiles) - 1;  // tile index within its slice, advanced per tile (no division)
     for (int i = 0; i < n_t; ++i) {
       const long long gt = g0 + i;
-      const int j = (int)(gt % tiles), ub = i & 1;
+      if (++j == tiles) j = 0;
+      const int ub = i & 1;
       if (i > 0 && j == 0) ++ls;
       // the next tile starts a slice: its M now, before this tile's statistics
       if (a.has_g && i + 1 < n_t && j == tiles - 1) build_m(ls + 1);
       wait(&u_full[ub], (uint32_t)(i >> 1) & 1u);
       __syncwarp();
       fence_after();
-      float x[64];
-      ld32(tmem + lrow + kFColU1 + 128 * ub + 64 * hf, x);
-      ld32(tmem + lrow + kFColU1 + 128 * ub + 64 * hf + 32, x + 32);
+      float x[TPP];
+#pragma unroll
+      for (int c = 0; c < TPP / 32; ++c) ld32(tmem + lrow + kFColU1 + 128 * ub + TPP * hf + 32 * c, x + 32 * c);
       wait_ld();
       fence_before();
       __syncwarp();
@@ -961,9 +982,9 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
       if constexpr (F32) {
         if (i + 1 < n_t) split_tile(i + 1);
       }
-      float part[12];  // per block kb: E, F, R at 3 kb
+      float part[3 * BPP];  // per block kb of the part: E, F, R at 3 kb
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {  // blocks 2 p and 2 p + 1 as fp32 pairs
+      for (int p = 0; p < BPP / 2; ++p) {  // blocks 2 p and 2 p + 1 as fp32 pairs
         float2 U[16], E, F, R;
         dct16_pair(x + 32 * p, x + 32 * p + 16, U);
         pair_sums(U, rad2, inv_tau, E, F, R);
@@ -975,6 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
         part[6 * p + 5] = R.y;
       }
       if constexpr (F32) {  // the halving butterfly, then the quarters' sums
+        static_assert(!F32 || BPP == 4, "the fp32 input's reduction takes 4 blocks per part");
         const float tot = warp_sum12(part, lane);
         float* rb = red + ((i & 1) * 2 + hf) * 48;
         if (!(lane & 1) && (lane >> 1) < 12) rb[wq * 12 + (lane >> 1)] = tot;
@@ -989,26 +1011,36 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_fwd_kernel(const __grid_
           a.lrate[blk] = R * 0.69314718055994531f / (16.0f * kD);
         }
       } else {
-        float* rb = red + ((i & 1) * 2 + hf) * (12 * kRedPitch);
+        float* rb = red + ((i & 1) * PARTS + hf) * (3 * BPP * kRedPitch);
 #pragma unroll
-        for (int q = 0; q < 12; ++q) rb[q * kRedPitch + v] = part[q];
+        for (int q = 0; q < 3 * BPP; ++q) rb[q * kRedPitch + v] = part[q];
         named_bar_sync(2 + hf, 128);
-        // One warp per half (channel quarter 3 or 2: not the SMSPs of the producer and MMA
-        // warps) finishes the sums: lane 8 kb + s adds v = 16 s .. 16 s + 15 of block kb.
-        if (wq == (hf ? 2 : 3)) {
-          const int kb = lane >> 3, sx = lane & 7;
+        // One warp per part (channel quarter 3 or 2: not the SMSPs of the producer and MMA
+        // warps) finishes the sums: LPB lanes per block, lane LPB kb + s adding the CPL
+        // channel frequencies v = CPL s .. CPL s + CPL - 1 of block kb.
+        if (wq == ((hf & 1) ? 2 : 3)) {
+          constexpr int LPB = 32 / BPP, CPL = kD / LPB;
+          const int kb = lane / LPB, sx = lane % LPB;
           float acc[3];
 #pragma unroll
           for (int c = 0; c < 3; ++c) {
-            const float4* src = reinterpret_cast<const float4*>(rb + (3 * kb + c) * kRedPitch + 16 * sx);
-            const float4 a0 = src[0], a1 = src[1], a2 = src[2], a3 = src[3];
-            acc[c] = (((a0.x + a0.y) + (a0.z + a0.w)) + ((a1.x + a1.y) + (a1.z + a1.w))) +
-                     (((a2.x + a2.y) + (a2.z + a2.w)) + ((a3.x + a3.y) + (a3.z + a3.w)));
+            const float4* src = reinterpret_cast<const float4*>(rb + (3 * kb + c) * kRedPitch + CPL * sx);
+            float4 q4[CPL / 4];
 #pragma unroll
-            for (int o = 1; o < 8; o <<= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
+            for (int w = 0; w < CPL / 4; ++w) q4[w] = src[w];
+            float s4[CPL / 4];
+#pragma unroll
+            for (int w = 0; w < CPL / 4; ++w) s4[w] = (q4[w].x + q4[w].y) + (q4[w].z + q4[w].w);
+#pragma unroll
+            for (int w2 = 1; w2 < CPL / 4; w2 <<= 1)
+#pragma unroll
+              for (int w = 0; w < CPL / 4; w += 2 * w2) s4[w] += s4[w + w2];
+            acc[c] = s4[0];
+#pragma unroll
+            for (int o = 1; o < LPB; o <<= 1) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
           }
           if (sx == 0) {
-            const long long blk = gt * 8 + 4 * hf + kb;
+            const long long blk = gt * 8 + BPP * hf + kb;
             a.lfreq[blk] = acc[0] > 0.0f ? acc[1] / acc[0] : 0.0f;
             a.lrate[blk] = acc[2] * 0.69314718055994531f / (16.0f * kD);
           }
@@ -1058,7 +1090,7 @@ cudaError_t launch_spectral_tmem(const KvGeom& k, int x_fp32, const void* x, con
     if (e != cudaSuccess) return e;
     const long long tiles = k.slices() * (k.T / kTile);
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-    kern<<<grid, kThreads, smem, st>>>(tmap, a);
+    kern<<<grid, x_fp32 ? FwdCfg<true>::THREADS : FwdCfg<false>::THREADS, smem, st>>>(tmap, a);
     return cudaGetLastError();
   }
   a.pieces = spectral_tmem_pieces(k);

@@ -190,6 +190,27 @@ def test_stats_forward_tile_ranges(gauged):
     _check(ref, lf, lr, tot)
 
 
+@pytest.mark.parametrize("want_grad", [False, True])
+def test_stats_large_magnitudes(want_grad):
+    """The rate sum takes log2 of products of four arguments 1 + |U| / tau; a product
+    overflows once |U| / tau passes about 2^32 and that block's sum is taken again two
+    arguments at a time.  A head slice at 1e9 (every block overflows), a channel at 3e8
+    (some coefficients of every block of its slice), a block at 1e7 (near the limit)
+    and ordinary blocks beside them, against the oracle."""
+    need_gpu()
+    L, B, H, T, d = 2, 1, 2, 512, 128
+    g = torch.Generator().manual_seed(33)
+    x = torch.randn((L, 2, B, H, T, d), generator=g)
+    x[0, 0, 0, 1] *= 1e9
+    x[1, 1, 0, 0, :, 5] *= 3e8
+    x[1, 0, 0, 1, 64:80] *= 1e7
+    x = x.to(torch.bfloat16).cuda().contiguous()
+    G = oracle_gauge(synth.gauge_params(L, H, 8, 16, sigma=0.1, seed=33))
+    lf, lr, tot, _ = run_stats(x, G, want_grad, False)
+    ref = sp.spectral_stats(bf16_np(x), G.cpu().numpy().astype(np.float64))
+    _check(ref, lf, lr, tot)
+
+
 @pytest.mark.parametrize("gauged", [True, False])
 def test_stats_fp32_input_tile_ranges(gauged):
     """fp32 input (already gauged, or with a g = 16 gauge applied in the kernel) takes the
