@@ -804,19 +804,25 @@ __global__ void __launch_bounds__(FwdCfg<F32>::THREADS, 1) spectral_fwd_kernel(c
 
   if (warp == 0) {
     if (lane == 0) {
-      int ls = -1, issued = 0;
+      int ls = -1, issued = 0, gq = 0;  // gq: G loads issued, for slices 0 .. gq - 1 of this range
+      const int n_sl = (int)((g0 + n_t - 1) / tiles - g0 / tiles) + 1;  // slices this range touches
+      // G of the range's q-th slice into buffer q & 1, once the workers have built the
+      // M of slice q - 2 from it
+      auto load_g = [&](int q) {
+        const int gb = q & 1;
+        wait(&g_empty[gb], ((uint32_t)(q >> 1) & 1u) ^ 1u);
+        int l, sk, b, h;
+        slice_coords(g0 / tiles + q, a.k, l, sk, b, h);
+        mbar_arrive_expect_tx(&g_full[gb], 8192);
+        bulk_g2s(gs + gb * 2048, a.G + gauge_set(l, sk, h, a.k) * 2048, 8192, &g_full[gb]);
+      };
       int j = (int)(g0 % tiles) - 1;  // tile index within its slice, advanced per tile
       for (int i = 0; i < n_t && !*abort_flag; ++i) {  // after a wait gave up, nothing more is issued
         const long long gt = g0 + i;
         if (++j == tiles) j = 0;
-        if (a.has_g && (i == 0 || j == 0)) {
+        if (a.has_g && (i == 0 || j == 0)) {  // a slice starts: its G and the next slice's are on the way
           ++ls;
-          const int gb = ls & 1;
-          wait(&g_empty[gb], ((uint32_t)(ls >> 1) & 1u) ^ 1u);
-          int l, sk, b, h;
-          slice_coords(gt / tiles, a.k, l, sk, b, h);
-          mbar_arrive_expect_tx(&g_full[gb], 8192);
-          bulk_g2s(gs + gb * 2048, a.G + gauge_set(l, sk, h, a.k) * 2048, 8192, &g_full[gb]);
+          while (gq <= ls + 1 && gq < n_sl && !*abort_flag) load_g(gq++);
         }
         const int s = i % NST;
         wait(&x_empty[s], ((uint32_t)(i / NST) & 1u) ^ 1u);
@@ -837,7 +843,7 @@ __global__ void __launch_bounds__(FwdCfg<F32>::THREADS, 1) spectral_fwd_kernel(c
         const int last = ((issued - 1 - s) / NST) * NST + s;
         mbar_wait(&x_full[s], (uint32_t)(last / NST) & 1u, a.status);
       }
-      for (int q = ls - 1 < 0 ? 0 : ls - 1; q <= ls; ++q) mbar_wait(&g_full[q & 1], (uint32_t)(q >> 1) & 1u, a.status);
+      for (int q = gq - 2 < 0 ? 0 : gq - 2; q < gq; ++q) mbar_wait(&g_full[q & 1], (uint32_t)(q >> 1) & 1u, a.status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -960,13 +966,19 @@ __global__ void __launch_bounds__(FwdCfg<F32>::THREADS, 1) spectral_fwd_kernel(c
     }
     int ls = 0;
     int j = (int)(g0 % tiles) - 1;  // tile index within its slice, advanced per tile (no division)
+    int j0 = j + 1;                 // the slice's first tile in this CTA's range
     for (int i = 0; i < n_t; ++i) {
       const long long gt = g0 + i;
       if (++j == tiles) j = 0;
       const int ub = i & 1;
-      if (i > 0 && j == 0) ++ls;
-      // the next tile starts a slice: its M now, before this tile's statistics
-      if (a.has_g && i + 1 < n_t && j == tiles - 1) build_m(ls + 1);
+      if (i > 0 && j == 0) {
+        ++ls;
+        j0 = 0;
+      }
+      // This warp's rows of the next slice's M, before this tile's statistics.  The
+      // token parts take their turns over the slice's last PARTS tiles, so that while
+      // one warp per SMSP builds, the other warps keep the arithmetic pipes busy.
+      if (a.has_g && i + (tiles - j) < n_t && j == max(tiles - 1 - hf, j0)) build_m(ls + 1);
       wait(&u_full[ub], (uint32_t)(i >> 1) & 1u);
       __syncwarp();
       fence_after();
