@@ -709,14 +709,17 @@ __global__ void __launch_bounds__(kThreads, 1) spectral_tmem_kernel(const __grid
 // cross into the next ones, each with its own gauge), instead of whole slices,
 // and U1^T is double-buffered in tensor memory so the GEMM of tile i + 1 runs
 // while the workers take tile i's token DCT and statistics.  M is double-buffered
-// too: the workers build the next slice's M before the current slice's last tile,
-// so the GEMM of the next slice's first tile overlaps that tile's statistics.
+// too: the workers build the next slice's M during the current slice's last tiles
+// (each token part at its own tile, from a G the producer loads a slice ahead), so
+// the GEMM of the next slice's first tile overlaps the current slice's statistics.
+// bf16 input: 16 worker warps, lane quarter = warp mod 4, token part (32 tokens) =
+// (warp - 2) / 4.  fp32 input: 8 worker warps, token halves of 64 tokens.
 // Tensor memory: [0,128) and [384,512) M (bf16 hi, lo), [128,256) and [256,384) U1^T.
 namespace {
 
 constexpr uint32_t kFColM0 = 0, kFColM1 = 384, kFColU1 = 128;
 __device__ __forceinline__ uint32_t fwd_mcol(int q) { return (q & 1) ? kFColM1 : kFColM0; }
-constexpr int kRedPitch = 132;  // [12][kRedPitch] partial sums of a tile half, by channel frequency v
+constexpr int kRedPitch = 132;  // [3 x blocks][kRedPitch] partial sums of a token part, by channel frequency v
 // bf16 input: a 4-stage ring of bf16 tiles, block sums finished in shared memory.  fp32 input:
 // a 2-stage ring of fp32 tiles (four 32-channel TMA boxes each), the current tile split by the
 // workers into bf16 hi and lo tiles (x = hi + lo to 2^-17), block sums by the warp butterfly.
