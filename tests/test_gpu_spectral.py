@@ -190,6 +190,22 @@ def test_stats_forward_tile_ranges(gauged):
     _check(ref, lf, lr, tot)
 
 
+@pytest.mark.parametrize("L,H,T", [(8, 8, 128), (4, 8, 256), (4, 4, 384)])
+def test_stats_forward_short_slices(L, H, T):
+    """Statistics only, with a gauge, on slices of one, two and three 128-token tiles:
+    fewer tiles than the forward kernel's four token parts, whose turns at building
+    the next slice's M then fall on the slice's first tile in the CTA's range.  256,
+    256 and 192 tiles over at most 148 CTAs, so ranges of one or two tiles cross slice
+    boundaries.  Every block against the oracle."""
+    need_gpu()
+    B, d = 2, 128
+    kv = synth.kv_cache(L, B, H, T, d, seed=9, device="cuda", n_outliers=2)
+    G = oracle_gauge(synth.gauge_params(L, H, 8, 16, sigma=0.1, seed=9))
+    lf, lr, tot, _ = run_stats(kv, G, False, False)
+    ref = sp.spectral_stats(bf16_np(kv), G.cpu().numpy().astype(np.float64))
+    _check(ref, lf, lr, tot)
+
+
 @pytest.mark.parametrize("want_grad", [False, True])
 def test_stats_large_magnitudes(want_grad):
     """The rate sum takes log2 of products of four arguments 1 + |U| / tau; a product
