@@ -1030,10 +1030,10 @@ __global__ void __launch_bounds__(FwdCfg<F32>::THREADS, 1) spectral_fwd_kernel(c
 #pragma unroll
         for (int q = 0; q < 3 * BPP; ++q) rb[q * kRedPitch + v] = part[q];
         named_bar_sync(2 + hf, 128);
-        // One warp per part (channel quarter 3 or 2: not the SMSPs of the producer and MMA
-        // warps) finishes the sums: LPB lanes per block, lane LPB kb + s adding the CPL
+        // One warp per part finishes the sums, the parts' reducers on different SMSPs
+        // (quarter 2 + hf mod 4): LPB lanes per block, lane LPB kb + s adding the CPL
         // channel frequencies v = CPL s .. CPL s + CPL - 1 of block kb.
-        if (wq == ((hf & 1) ? 2 : 3)) {
+        if (wq == ((2 + hf) & 3)) {
           constexpr int LPB = 32 / BPP, CPL = kD / LPB;
           const int kb = lane / LPB, sx = lane % LPB;
           float acc[3];
