@@ -12,8 +12,8 @@
 // the codes remains.
 //
 // Two kernels (flash decoding):
-//   partial: one CTA per (layer, batch, KV head, 256-token chunk) and all query
-//     heads of the GQA group.  The chunk's key and value codes, steps and zero
+//   partial: one CTA per (layer, batch, KV head, run of kCpc 128-token chunks)
+//     and all query heads of the GQA group.  Each chunk's key and value codes, steps and zero
 //     points are staged in shared memory with coalesced 16-byte loads.  Both
 //     contractions run on the warp-level tensor cores (mma.sync m16n8k16,
 //     fp16 operands, fp32 accumulation), one MMA per 16 x 16 range block, with
@@ -25,7 +25,7 @@
 //               the block's value codes transposed, B = the softmax weights as
 //               fp16 hi + lo terms (scaled by 2^12);
 //     the block's step and zero point apply to each MMA result.  Writes (max,
-//     sum, o[d]) per (query head, chunk);
+//     sum, o[d]) per (query head, run of chunks);
 //   combine: per (layer, batch, query head): merges the chunks' partials with
 //     the usual rescaling, divides by the total, applies G_V^T per group.
 #include "cg_kernels.cuh"
@@ -34,8 +34,8 @@ namespace cg {
 
 namespace {
 
-constexpr int kChunk = 256;  // tokens per chunk
-constexpr int kCpc = 4;      // chunks per CTA (one partial per CTA)
+constexpr int kChunk = 128;  // tokens per chunk (about 46 KB of shared memory per CTA at d = 128: 4 CTAs per SM)
+constexpr int kCpc = 8;      // chunks per CTA (one partial per CTA)
 constexpr int kAttnThreads = 256;
 
 // Asynchronous global -> shared copies (16 bytes bypassing L1, or 4 bytes),
@@ -316,10 +316,11 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
     }
     __syncthreads();
 
-    // ---- softmax over the chunk, thread = token ----
+    // ---- softmax over the chunk, thread = token (threads past the chunk only reduce) ----
     {
       const int t = tid;
       const bool live = t < ntok;
+      const bool row = t < kChunk;  // threads past the chunk take part in the reductions only
       float sj[GQ];
   #pragma unroll
       for (int j = 0; j < GQ; ++j) {
@@ -344,11 +345,13 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
         const float ps = pj * kPScale;
         const __half hi = __float2half_rn(ps);
         const __half lo = __float2half_rn(ps - __half2float(hi));
-        pb[j * kChunk + t] = __half_as_ushort(hi);  // lo terms: column 4 + j (GQ <= 4) or 8 + j
-        pb[(NT == 2 ? 8 + j : 4 + j) * kChunk + t] = __half_as_ushort(lo);
+        if (row) {
+          pb[j * kChunk + t] = __half_as_ushort(hi);  // lo terms: column 4 + j (GQ <= 4) or 8 + j
+          pb[(NT == 2 ? 8 + j : 4 + j) * kChunk + t] = __half_as_ushort(lo);
+        }
       }
       if constexpr (NT == 1) {  // unused columns of the tile are zero
-        for (int j = GQ; j < 4; ++j) {
+        for (int j = GQ; j < 4 && row; ++j) {
           pb[j * kChunk + t] = 0;
           pb[(4 + j) * kChunk + t] = 0;
         }
@@ -359,7 +362,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
         float s16 = ls[j];  // per 16-token block (half a warp), then per warp
   #pragma unroll
         for (int o = 8; o >= 1; o >>= 1) s16 += __shfl_xor_sync(0xffffffffu, s16, o);
-        if ((lane & 15) == 0) psum[(t >> 4) * GQ + j] = s16;
+        if ((lane & 15) == 0 && row) psum[(t >> 4) * GQ + j] = s16;
         const float s32 = s16 + __shfl_xor_sync(0xffffffffu, s16, 16);
         if (lane == 0) red[warp * GQ + j] = s32;
       }

@@ -4,11 +4,12 @@ fp64 (G^T (s q + z)) and runs plain softmax attention; the device folds the
 gauge into the query and the output.  Tolerance: per (layer, batch, query head)
 output vector, norm-relative 1e-4 (fp32 sums over up to 4096 tokens).
 
-Launch geometry: one CTA per (layer, batch, KV head, 256-token chunk), then one
-per (layer, batch, query head) for the merge; the cases cover one chunk, a last
-chunk of 16 tokens, several chunks, a layer range inside the cache, every GQA
-group size and the 8B-shaped cache (32 layers, 32 query heads over 8 KV heads,
-4096 tokens: 4096 CTAs) on sampled slices."""
+Launch geometry: one CTA per (layer, batch, KV head, run of eight 128-token
+chunks), then one per (layer, batch, query head) for the merge; the cases cover
+one chunk, a last chunk of 16 or 112 tokens, several chunks in one CTA, a layer
+range inside the cache, every GQA group size and the 8B-shaped cache (32 layers,
+32 query heads over 8 KV heads, 4096 tokens: 1024 CTAs, four partials merged per
+query head) on sampled slices."""
 import numpy as np
 import pytest
 import torch
