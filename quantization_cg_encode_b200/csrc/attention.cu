@@ -12,7 +12,7 @@
 // the codes remains.
 //
 // Two kernels (flash decoding):
-//   partial: one CTA per (layer, batch, KV head, run of kCpc 128-token chunks)
+//   partial: one CTA per (layer, batch, KV head, run of cpc 128-token chunks)
 //     and all query heads of the GQA group.  Each chunk's key and value codes, steps and zero
 //     points are staged in shared memory with coalesced 16-byte loads.  Both
 //     contractions run on the warp-level tensor cores (mma.sync m16n8k16,
@@ -35,7 +35,7 @@ namespace cg {
 namespace {
 
 constexpr int kChunk = 128;  // tokens per chunk (about 46 KB of shared memory per CTA at d = 128: 4 CTAs per SM)
-constexpr int kCpc = 8;      // chunks per CTA (one partial per CTA)
+constexpr int kMaxCpc = 8;   // chunks per CTA (one partial per CTA) at most; the launcher picks 1, 2, 4 or 8
 constexpr int kAttnThreads = 256;
 
 // Asynchronous global -> shared copies (16 bytes bypassing L1, or 4 bytes),
@@ -67,7 +67,7 @@ __device__ __forceinline__ uint32_t nib_hi_pair(uint32_t w) {
 }  // namespace
 
 // partial[l][b][hq][split] = {m, l, o[D]} in gauge coordinates, over the token
-// chunks [split kCpc, split kCpc + kCpc) of one (layer, batch, KV head).
+// chunks [split cpc, split cpc + cpc) of one (layer, batch, KV head).
 //
 // MMA columns: for GQ <= 4 one N = 8 tile holds the hi terms of heads 0..3 in
 // columns 0..3 and the lo terms in 4..7 (heads >= GQ are zero); for GQ = 8 a
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c = lane & 3;
   const int n_tc = (a.n_tokens + kChunk - 1) / kChunk;  // token chunks
-  const int c0 = split * kCpc, c1 = min(n_tc, c0 + kCpc);
+  const int c0 = split * a.cpc, c1 = min(n_tc, c0 + a.cpc);
   const long long slice_k = (((long long)l * 2 + 0) * a.k.B + b) * a.k.H + h;
   const long long slice_v = (((long long)l * 2 + 1) * a.k.B + b) * a.k.H + h;
   const long long slice_bytes = (long long)a.k.T * D * BITS / 8;
@@ -565,7 +565,7 @@ cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {
   auto kern = attn_partial_kernel<D, BITS, GQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.n_chunks, a.k.B * a.k.H, a.n_layers);  // one CTA per split of kCpc chunks
+  dim3 grid(a.n_chunks, a.k.B * a.k.H, a.n_layers);  // one CTA per split of cpc chunks
   kern<<<grid, kAttnThreads, smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -609,8 +609,15 @@ uint64_t attn_workspace_bytes(const KvGeom& k, int hq, int n_layers, int n_token
   return (uint64_t)n_layers * k.B * hq * chunks * (k.d + 2) * sizeof(float);
 }
 
-cudaError_t launch_decode_attention(AttnArgs a, cudaStream_t st) {
-  a.n_chunks = ((a.n_tokens + kChunk - 1) / kChunk + kCpc - 1) / kCpc;  // partials per (layer, batch, query head)
+cudaError_t launch_decode_attention(AttnArgs a, int num_sms, cudaStream_t st) {
+  // Chunks per CTA: as many as keep at least six CTAs per SM (four are resident
+  // at a time), so that small calls still fill the GPU and large ones run and
+  // merge fewer partials.
+  const int n_tc = (a.n_tokens + kChunk - 1) / kChunk;
+  const long long heads = (long long)a.n_layers * a.k.B * a.k.H;
+  a.cpc = kMaxCpc;
+  while (a.cpc > 1 && heads * ((n_tc + a.cpc - 1) / a.cpc) < 6LL * num_sms) a.cpc >>= 1;
+  a.n_chunks = (n_tc + a.cpc - 1) / a.cpc;  // partials per (layer, batch, query head)
   return a.k.d == 128 ? attn_bits<128>(a, st) : attn_bits<64>(a, st);
 }
 

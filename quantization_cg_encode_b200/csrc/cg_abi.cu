@@ -313,7 +313,7 @@ cg_status cg_decode_attention(const cg_kv_desc* kv, const cg_codec_desc* codec, 
   a.G = G_dev;
   a.out = out_dev;
   a.partial = (float*)workspace_dev;
-  return from_cuda(launch_decode_attention(a, (cudaStream_t)stream));
+  return from_cuda(launch_decode_attention(a, num_sms(), (cudaStream_t)stream));
 }
 
 cg_status cg_spectral_workspace_size(const cg_kv_desc* kv, const cg_stats_desc* st, int32_t want_grad, uint64_t* bytes) {

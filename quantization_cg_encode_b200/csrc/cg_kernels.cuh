@@ -69,7 +69,8 @@ struct AttnArgs {
   int hq;                 // query heads (a multiple of H)
   int n_tokens;           // attend to tokens [0, n_tokens), a multiple of 16
   int l0, n_layers;       // layers [l0, l0 + n_layers)
-  int n_chunks;           // set by the launcher
+  int n_chunks;           // partials per (layer, batch, query head): set by the launcher
+  int cpc;                // 128-token chunks per CTA: set by the launcher
   float scale;            // score scale (1/sqrt(d) by default)
   const uint16_t* q;      // bf16 [n_layers][B][hq][d]
   const uint8_t* codes;   // whole cache, block-uniform 16 x 16 ranges
@@ -80,7 +81,7 @@ struct AttnArgs {
   float* partial;         // workspace
 };
 uint64_t attn_workspace_bytes(const KvGeom& k, int hq, int n_layers, int n_tokens);
-cudaError_t launch_decode_attention(AttnArgs a, cudaStream_t st);
+cudaError_t launch_decode_attention(AttnArgs a, int num_sms, cudaStream_t st);
 
 // 2-D TMA tensor map over a row-major bf16 [rows][cols] array (box_cols x
 // box_rows boxes, 128-byte swizzle); `out` points to a CUtensorMap.
