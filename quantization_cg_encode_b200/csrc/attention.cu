@@ -12,7 +12,7 @@
 // the codes remains.
 //
 // Two kernels (flash decoding):
-//   partial: one CTA per (layer, batch, KV head, run of cpc 128-token chunks)
+//   partial: one CTA per (layer, batch, KV head, run of cpc chunks of 128 or 256 tokens)
 //     and all query heads of the GQA group.  Each chunk's key and value codes, steps and zero
 //     points are staged in shared memory with coalesced 16-byte loads.  Both
 //     contractions run on the warp-level tensor cores (mma.sync m16n8k16,
@@ -34,7 +34,10 @@ namespace cg {
 
 namespace {
 
-constexpr int kChunk = 128;  // tokens per chunk (about 46 KB of shared memory per CTA at d = 128: 4 CTAs per SM)
+// Tokens per chunk: 128 (about 46 KB of shared memory per CTA at d = 128: four CTAs
+// per SM) or 256 (85 KB: two per SM, half the phase synchronisations per token),
+// chosen by the launcher.
+constexpr int kSmallChunk = 128, kLargeChunk = 256;
 constexpr int kMaxCpc = 8;   // chunks per CTA (one partial per CTA) at most; the launcher picks 1, 2, 4 or 8
 constexpr int kAttnThreads = 256;
 
@@ -76,7 +79,7 @@ __device__ __forceinline__ uint32_t nib_hi_pair(uint32_t w) {
 // A CTA's chunks stream through two shared-memory stages (cp.async: the next
 // chunk's codes, steps and zero points load while the current one computes)
 // and are merged with the online softmax rescaling.
-template <int D, int BITS, int GQ>
+template <int D, int BITS, int GQ, int kChunk>
 __global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(AttnArgs a) {
   constexpr int NG = D / 16;
   constexpr int BLK = 32 * BITS;                 // bytes of one 16 x 16 range block
@@ -551,7 +554,7 @@ __global__ void __launch_bounds__(D) attn_combine_kernel(AttnArgs a) {
 
 namespace {
 
-template <int D, int BITS, int GQ>
+template <int D, int BITS, int GQ, int kChunk>
 cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {
   constexpr int NG = D / 16;
   constexpr int CODE_BYTES = kChunk * D * BITS / 8;
@@ -562,7 +565,7 @@ cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {
   const int smem_floats = GQ * D + GQ * NG + 8 + kChunk * GQ + NBLK * GQ + 8 * GQ + 8 + 32 + 2 * GQ * D + NBLK * GQ +
                           NG * NT * 64;
   const size_t smem = 2 * (size_t)STAGE + 4 * (size_t)smem_floats + 2 * (size_t)NCOL * kChunk;
-  auto kern = attn_partial_kernel<D, BITS, GQ>;
+  auto kern = attn_partial_kernel<D, BITS, GQ, kChunk>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_chunks, a.k.B * a.k.H, a.n_layers);  // one CTA per split of cpc chunks
@@ -582,10 +585,10 @@ cudaError_t attn_launch(const AttnArgs& a, cudaStream_t st) {
 template <int D, int BITS>
 cudaError_t attn_gq(const AttnArgs& a, cudaStream_t st) {
   switch (a.hq / a.k.H) {
-    case 1: return attn_launch<D, BITS, 1>(a, st);
-    case 2: return attn_launch<D, BITS, 2>(a, st);
-    case 4: return attn_launch<D, BITS, 4>(a, st);
-    case 8: return attn_launch<D, BITS, 8>(a, st);
+    case 1: return a.chunk == kLargeChunk ? attn_launch<D, BITS, 1, kLargeChunk>(a, st) : attn_launch<D, BITS, 1, kSmallChunk>(a, st);
+    case 2: return a.chunk == kLargeChunk ? attn_launch<D, BITS, 2, kLargeChunk>(a, st) : attn_launch<D, BITS, 2, kSmallChunk>(a, st);
+    case 4: return a.chunk == kLargeChunk ? attn_launch<D, BITS, 4, kLargeChunk>(a, st) : attn_launch<D, BITS, 4, kSmallChunk>(a, st);
+    case 8: return a.chunk == kLargeChunk ? attn_launch<D, BITS, 8, kLargeChunk>(a, st) : attn_launch<D, BITS, 8, kSmallChunk>(a, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -605,19 +608,26 @@ cudaError_t attn_bits(const AttnArgs& a, cudaStream_t st) {
 }  // namespace
 
 uint64_t attn_workspace_bytes(const KvGeom& k, int hq, int n_layers, int n_tokens) {
-  const uint64_t chunks = (uint64_t)(n_tokens + kChunk - 1) / kChunk;
+  const uint64_t chunks = (uint64_t)(n_tokens + kSmallChunk - 1) / kSmallChunk;  // at most one partial per chunk
   return (uint64_t)n_layers * k.B * hq * chunks * (k.d + 2) * sizeof(float);
 }
 
 cudaError_t launch_decode_attention(AttnArgs a, int num_sms, cudaStream_t st) {
-  // Chunks per CTA: as many as keep at least six CTAs per SM (four are resident
-  // at a time), so that small calls still fill the GPU and large ones run and
-  // merge fewer partials.
-  const int n_tc = (a.n_tokens + kChunk - 1) / kChunk;
+  // A call whose CTAs of four 256-token chunks fit in one wave (two per SM) runs
+  // them.  Larger calls take 128-token chunks, four CTAs per SM, as many per CTA
+  // as keep at least six CTAs per SM, so that they run and merge fewer partials.
   const long long heads = (long long)a.n_layers * a.k.B * a.k.H;
-  a.cpc = kMaxCpc;
-  while (a.cpc > 1 && heads * ((n_tc + a.cpc - 1) / a.cpc) < 6LL * num_sms) a.cpc >>= 1;
-  a.n_chunks = (n_tc + a.cpc - 1) / a.cpc;  // partials per (layer, batch, query head)
+  const int n_large = (a.n_tokens + kLargeChunk - 1) / kLargeChunk;
+  if (heads * ((n_large + 3) / 4) <= 2LL * num_sms) {
+    a.chunk = kLargeChunk;
+    a.cpc = 4;
+  } else {
+    a.chunk = kSmallChunk;
+    const int n_small = (a.n_tokens + kSmallChunk - 1) / kSmallChunk;
+    a.cpc = kMaxCpc;
+    while (a.cpc > 1 && heads * ((n_small + a.cpc - 1) / a.cpc) < 6LL * num_sms) a.cpc >>= 1;
+  }
+  a.n_chunks = ((a.n_tokens + a.chunk - 1) / a.chunk + a.cpc - 1) / a.cpc;  // partials per (layer, batch, query head)
   return a.k.d == 128 ? attn_bits<128>(a, st) : attn_bits<64>(a, st);
 }
 

@@ -70,7 +70,8 @@ struct AttnArgs {
   int n_tokens;           // attend to tokens [0, n_tokens), a multiple of 16
   int l0, n_layers;       // layers [l0, l0 + n_layers)
   int n_chunks;           // partials per (layer, batch, query head): set by the launcher
-  int cpc;                // 128-token chunks per CTA: set by the launcher
+  int chunk;              // tokens per chunk, 128 or 256: set by the launcher
+  int cpc;                // chunks per CTA: set by the launcher
   float scale;            // score scale (1/sqrt(d) by default)
   const uint16_t* q;      // bf16 [n_layers][B][hq][d]
   const uint8_t* codes;   // whole cache, block-uniform 16 x 16 ranges
