@@ -4,12 +4,14 @@ fp64 (G^T (s q + z)) and runs plain softmax attention; the device folds the
 gauge into the query and the output.  Tolerance: per (layer, batch, query head)
 output vector, norm-relative 1e-4 (fp32 sums over up to 4096 tokens).
 
-Launch geometry: one CTA per (layer, batch, KV head, run of eight 128-token
-chunks), then one per (layer, batch, query head) for the merge; the cases cover
+Launch geometry: one CTA per (layer, batch, KV head, run of chunks), then one
+per (layer, batch, query head) for the merge; the cases cover
 one chunk, a last chunk of 16 or 112 tokens, several chunks in one CTA, a layer
 range inside the cache, every GQA group size and the 8B-shaped cache (32 layers,
 32 query heads over 8 KV heads, 4096 tokens: 1024 CTAs, four partials merged per
-query head) on sampled slices."""
+query head) on sampled slices.  The launcher picks the chunk size: the small cases
+fit one wave of 256-token chunks; the 8B-shaped cache and a ragged 10-layer call
+(two 128-token chunks per CTA, a last chunk of 80 tokens) take 128-token chunks."""
 import numpy as np
 import pytest
 import torch
@@ -84,3 +86,29 @@ def test_decode_attention_8b_shaped_cache_sampled():
                                     Gn[l:l + 1, :, h:h + 1], 4)           # [1, 2, B, 1, T, d]
         ref = oa.softmax_attention(qn[l, :, 4 * h:4 * h + 4], x[0, 0], x[0, 1], float(np.float32(scale)))
         _close(got[l, :, 4 * h:4 * h + 4], ref, "8B slice %s" % ((l, h),))
+
+
+def test_decode_attention_small_chunks_ragged_sampled():
+    """A call too large for one wave of 256-token chunks: 10 layers x 2 batches x 8 KV
+    heads over 2000 of 2048 tokens takes 128-token chunks, two per CTA (1280 CTAs),
+    with a last chunk of 80 tokens; sampled (layer, batch, KV head) slices against
+    the oracle."""
+    need_gpu()
+    L, B, H, T, d, Hq, n = 10, 2, 8, 2048, 128, 32, 2000
+    kv, G, codec, codes, scales, zeros = _encoded(L, B, H, T, d, 4, seed=12)
+    q = torch.randn((L, B, Hq, d), generator=torch.Generator().manual_seed(6)).to(torch.bfloat16).cuda()
+    scale = 1.0 / np.sqrt(d)
+    got = _attend(kv, G, codec, codes, scales, zeros, q, n, 0, scale)
+    c, s, z = block_uniform_np(codes, scales, zeros, kv.shape, codec)
+    Gn = G.cpu().numpy().astype(np.float64)
+    qn = bf16_np(q)
+    rng = np.random.default_rng(7)
+    for _ in range(3):
+        l, h = int(rng.integers(L)), int(rng.integers(H))
+        x = oc.decode_block_uniform(c[l:l + 1, :, :, h:h + 1], z[l:l + 1, :, :, h:h + 1].view(np.float16).astype(np.float64),
+                                    s[l:l + 1, :, :, h:h + 1].view(np.float16).astype(np.float64),
+                                    Gn[l:l + 1, :, h:h + 1], 4)           # [1, 2, B, 1, T, d]
+        for b in range(B):
+            ref = oa.softmax_attention(qn[l, b:b + 1, 4 * h:4 * h + 4], x[0, 0, b:b + 1, :, :n], x[0, 1, b:b + 1, :, :n],
+                                       float(np.float32(scale)))
+            _close(got[l, b:b + 1, 4 * h:4 * h + 4], ref, "slice %s" % ((l, b, h),))
