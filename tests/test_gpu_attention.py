@@ -6,7 +6,7 @@ output vector, norm-relative 1e-4 (fp32 sums over up to 4096 tokens).
 
 Launch geometry: one CTA per (layer, batch, KV head, run of chunks), then one
 per (layer, batch, query head) for the merge; the cases cover
-one chunk, a last chunk of 16 or 112 tokens, several chunks in one CTA, a layer
+one chunk, a last chunk of 16 or 240 tokens, several chunks in one CTA, a layer
 range inside the cache, every GQA group size and the 8B-shaped cache (32 layers,
 32 query heads over 8 KV heads, 4096 tokens: 1024 CTAs, four partials merged per
 query head) on sampled slices.  The launcher picks the chunk size: the small cases
